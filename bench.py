@@ -1,0 +1,469 @@
+"""Benchmark of the sparse MoE FFN layer forward on B200 (sm_100a).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+One step = one moe_forward over a batch of T tokens of the named workload
+(default: the Hy4-shape prefill layer, T=4096, H=6144, E=256 top-8 + 1 shared,
+I=2048, bf16) with inputs resident in HBM.  Under torchrun each rank runs the
+same layer on its own batch (data-parallel replicas, no collective on the data
+path: weak scaling); the reported time is the max over ranks.
+
+Printed (rank 0, one JSON line): tokens/s, the layer's roofline fraction, the
+dominant kernel's roofline record (CUDA-event duration inside the timed
+region), an end-to-end figure through host buffers, SM clocks sampled during
+the timed region, our kernel launch count and the CPU oracle baseline.
+``--impl reference`` times the CPU oracle instead (the reference arm).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from sparse_moe_layer_06_b200.workloads import CONFIGS, make_inputs, make_x, sample_tokens  # noqa
+
+METRIC = "MoE-layer tokens/s and % of roofline (TFLOP/s or HBM GB/s) on 1 B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+GEMM_SOURCES = ["sparse_moe_layer_06_b200/csrc/gemm_sm100.cuh",
+                "sparse_moe_layer_06_b200/csrc/ptx.cuh"]
+
+
+# ------------------------------------------------------------------ helpers
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def layer_counts(cfg, idx_cpu):
+    """Algorithmic FLOPs and bytes of one layer forward, from the actual routing."""
+    T, H, E, I, k, S = cfg.T, cfg.H, cfg.E, cfg.I, cfg.top_k, cfg.num_shared
+    b = 2 if cfg.dtype == torch.bfloat16 else 4
+    touched = int((torch.bincount(idx_cpu.reshape(-1).long(), minlength=E) > 0).sum())
+    flops = T * (2 * H * E + (k + S) * 6 * H * I)
+    bytes_ = (touched + S) * 3 * I * H * b + E * H * b + 2 * T * H * b
+    return flops, bytes_, touched
+
+
+def gate_up_counts(cfg, touched):
+    """Algorithmic FLOPs / bytes of one launch of the grouped gate/up GEMM:
+    gate+up weights of every touched expert (+ shared), the permuted token rows
+    and x (shared expert) read once, h written once."""
+    T, H, I, k, S = cfg.T, cfg.H, cfg.I, cfg.top_k, cfg.num_shared
+    rows = T * (k + S)
+    flops = 2 * 2 * rows * H * I
+    bytes_ = (touched + S) * 2 * I * H * 2 + rows * H * 2 + rows * I * 2
+    return flops, bytes_
+
+
+def down_counts(cfg, touched):
+    """One launch of the grouped down GEMM + weighted scatter-add: down weights
+    of every touched expert (+ shared), h read once, the fp32 accumulator read
+    and written once per token."""
+    T, H, I, k, S = cfg.T, cfg.H, cfg.I, cfg.top_k, cfg.num_shared
+    rows = T * (k + S)
+    flops = 2 * rows * H * I
+    bytes_ = (touched + S) * I * H * 2 + rows * I * 2 + 2 * T * H * 4
+    return flops, bytes_
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for rel in GEMM_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch recorded from an ncu capture of this kernel
+    (profiles/ncu_traffic.txt); None if absent or the kernel source changed."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    want = source_hash()
+    for line in open(path):
+        if line.startswith("#") or not line.strip():
+            continue
+        f = dict(kv.split("=", 1) for kv in line.split() if "=" in kv)
+        if f.get("kernel") == kernel and f.get("workload") == workload and \
+                f.get("source_hash") == want:
+            return int(float(f["bytes_per_launch"]))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms; summary() keeps only the
+    samples taken inside a given wall-clock window (the timed region)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.samples = []  # (wall time, fields)
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return self
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.thread:
+                self.thread.join(timeout=2)
+
+    def summary(self, t0: float, t1: float):
+        rows = [r for (t, r) in self.samples if t0 <= t <= t1]
+        mine = [r for r in rows if r[0] == str(self.gpu)] or rows
+        if not mine:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples in window"],
+                    "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in mine if num(r[1]) is not None]
+        smax = [num(r[2]) for r in mine if num(r[2]) is not None]
+        pw = [num(r[3]) for r in mine if num(r[3]) is not None]
+        reasons = sorted({self.REASONS[i] for r in mine for i in range(4)
+                          if r[5 + i].lower() in ("active", "1")})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(pw) if pw else None,
+                "reasons": reasons, "samples": len(mine)}
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+
+def oracle_baseline(cfg, cpu_inp, budget_s=12.0, max_tokens=256):
+    """Time the CPU oracle (as it stands) on a seeded token sample of the same
+    workload: batches of tokens until ~budget_s of work.  Returns a dict."""
+    import oracle
+    order = sample_tokens(cfg.T, min(cfg.T, max_tokens), seed=1)
+    done = 0
+    t0 = time.perf_counter()
+    batch = max(1, oracle.num_threads())
+    while done < len(order):
+        toks = order[done:done + batch]
+        oracle.forward(cpu_inp["x"], cpu_inp["gate_w"], cpu_inp["expert_w"], cpu_inp["shared_w"],
+                       cfg.top_k, cfg.routed_scale, cfg.clip_limit,
+                       logit_bias=cpu_inp["logit_bias"], tokens=toks)
+        done += len(toks)
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": done / dt, "unit": "tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{done} seeded tokens of the {cfg.name} batch (T={cfg.T}), "
+                      f"full layer per token, fp64, {dt:.1f} s"}
+
+
+def cpu_inputs(inp):
+    return {k: (v.detach().cpu() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args, cfg, rank, world):
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    torch.manual_seed(0)
+    inp = make_inputs(cfg, seed=0, device="cpu") if cfg.T * cfg.H * cfg.E < 1 << 33 else None
+    if inp is None:
+        inp = cpu_inputs(make_inputs(cfg, seed=0, device="cuda"))
+        torch.cuda.empty_cache()
+    order = sample_tokens(cfg.T, cfg.T, seed=1)
+    # calibrate tokens per step so that warmup+steps fit in ~150 s
+    t0 = time.perf_counter()
+    oracle.forward(inp["x"], inp["gate_w"], inp["expert_w"], inp["shared_w"], cfg.top_k,
+                   cfg.routed_scale, cfg.clip_limit, logit_bias=inp["logit_bias"],
+                   tokens=order[:1])
+    per_tok = max(1e-6, time.perf_counter() - t0)
+    n_steps = args.steps + args.warmup
+    per_step = max(1, min(cfg.T, int(150.0 / n_steps / per_tok * max(1, oracle.num_threads()))))
+    times = []
+    cursor = 0
+    for s in range(n_steps):
+        toks = [order[(cursor + i) % cfg.T] for i in range(per_step)]
+        cursor += per_step
+        t0 = time.perf_counter()
+        oracle.forward(inp["x"], inp["gate_w"], inp["expert_w"], inp["shared_w"], cfg.top_k,
+                       cfg.routed_scale, cfg.clip_limit, logit_bias=inp["logit_bias"],
+                       tokens=toks)
+        if s >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = per_step * len(times) / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "top_k": cfg.top_k,
+                   "I": cfg.I, "num_shared": cfg.num_shared, "tokens_per_step": per_step},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"{per_step} seeded tokens of the {cfg.name} batch per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=600)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="hy4_prefill", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override T of the workload (smaller cases for profiling)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="override E of the workload (smaller cases for profiling)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = CONFIGS[args.config]
+    if args.tokens is not None or args.experts is not None:
+        from dataclasses import replace
+        cfg = replace(cfg, T=args.tokens or cfg.T, E=args.experts or cfg.E,
+                      name=f"{cfg.name}_T{args.tokens or cfg.T}_E{args.experts or cfg.E}")
+
+    if args.impl == "reference":
+        return run_reference(args, cfg, rank, world)
+
+    from sparse_moe_layer_06_b200 import moe
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    # identical weights on every rank, a different token batch per rank
+    inp = make_inputs(cfg.with_tokens(1), seed=0, device=dev)
+    inp["x"] = make_x(cfg, seed=1000 * rank, device=dev)
+    if cfg.skew_bias:
+        from sparse_moe_layer_06_b200.workloads import skew_logit_bias
+        inp["logit_bias"] = skew_logit_bias(cfg.E).to(dev)
+    p = moe.MoEProblem.from_config(cfg)
+    ws = moe.alloc_workspace(p, moe.MOE_CALL_FORWARD, device=dev)
+    out = torch.empty(cfg.T, cfg.H, dtype=cfg.dtype, device=dev)
+    idx = torch.empty(cfg.T, cfg.top_k, dtype=torch.int32, device=dev)
+    w = torch.empty(cfg.T, cfg.top_k, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        moe.moe_forward(p, inp["x"], inp["gate_w"], inp["logit_bias"], inp["expert_w"],
+                        inp["shared_w"], out, idx, w, ws, stream)
+
+    gpu_index = local if torch.cuda.device_count() > 1 else 0
+    clocks = ClockSampler(gpu_index).start()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if moe.moe_read_device_status(ws) != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    # ---------------- timed region (device time, CUDA events, max over ranks)
+    moe.moe_profile_start(args.steps * 16 + 64)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = moe.moe_launch_count()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    wall0 = time.time()
+    ev1.synchronize()
+    wall1 = time.time()
+    launches = moe.moe_launch_count() - launches0
+    if dist:
+        dist.barrier()
+    kernel_times = moe.moe_profile_stop()
+    clocks.stop()
+    ms = ev0.elapsed_time(ev1)
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    status = moe.moe_read_device_status(ws)
+    ms_per_step = ms / args.steps
+
+    # ---------------- end to end: host buffers, copies inside the timed region
+    x_host = inp["x"].cpu().pin_memory()
+    out_host = torch.empty(cfg.T, cfg.H, dtype=cfg.dtype).pin_memory()
+    x_dev = torch.empty_like(inp["x"])
+    for _ in range(3):
+        x_dev.copy_(x_host, non_blocking=True)
+        moe.moe_forward(p, x_dev, inp["gate_w"], inp["logit_bias"], inp["expert_w"],
+                        inp["shared_w"], out, idx, w, ws, stream)
+        out_host.copy_(out, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        moe.moe_forward(p, x_dev, inp["gate_w"], inp["logit_bias"], inp["expert_w"],
+                        inp["shared_w"], out, idx, w, ws, stream)
+        out_host.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+        dist.barrier()
+
+    if rank != 0:
+        if dist:
+            dist.destroy_process_group()
+        return 0
+
+    # ---------------- derived numbers
+    peaks, peak_kind = read_peaks()
+    hbm_peak = float(peaks["hbm_gbs"])
+    tf_peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    idx_cpu = idx.cpu()
+    flops, bytes_, touched = layer_counts(cfg, idx_cpu)
+    t_s = ms_per_step / 1e3
+    tokens_per_s = world * cfg.T / t_s
+    roof_t = max(flops / (tf_peak * 1e12), bytes_ / (hbm_peak * 1e9))
+    layer_frac = roof_t / t_s
+    roof_t_nominal = max(flops / 2250e12, bytes_ / 8000e9)
+
+    per_kernel = {k: {"launches": v[0], "ms_per_launch": v[1] / max(1, v[0]),
+                      "share": v[1] / max(1e-9, sum(x[1] for x in kernel_times.values()))}
+                  for k, v in kernel_times.items()}
+    dominant = max(kernel_times, key=lambda k: kernel_times[k][1])
+    dom_ms = kernel_times[dominant][1] / max(1, kernel_times[dominant][0])
+    if dominant == "expert_down_combine_gemm":
+        kf, kb = down_counts(cfg, touched)
+    else:
+        kf, kb = gate_up_counts(cfg, touched)
+    dom_s = dom_ms / 1e3
+    t_hbm = kb / (hbm_peak * 1e9)
+    t_tc = kf / (tf_peak * 1e12)
+    if t_hbm >= t_tc:
+        roof = {"bound": "hbm", "achieved": kb / dom_s / 1e9, "peak": hbm_peak, "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": kf / dom_s / 1e12, "peak": tf_peak,
+                "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = ncu_traffic(dominant, cfg.name)
+    roof["kernel"] = dominant
+    roof["algorithmic"] = {"bytes": kb, "flops": kf}
+    roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" \
+        else "fallback"
+
+    cpu_base = None
+    if not args.no_cpu_baseline and world == 1:
+        import oracle
+        oracle.build()
+        cpu_inp = cpu_inputs(inp)
+        cpu_base = oracle_baseline(cfg, cpu_inp)
+
+    h2d = cfg.T * cfg.H * x_host.element_size()
+    d2h = cfg.T * cfg.H * out_host.element_size()
+    line = {
+        "metric": METRIC,
+        "value": tokens_per_s,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if cfg.dtype == torch.bfloat16 else "f32",
+        "data": "synthetic (seeded N(0,1) tokens, N(0,0.006) weights; random init)",
+        "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E,
+                   "top_k": cfg.top_k, "I": cfg.I, "num_shared": cfg.num_shared,
+                   "global_batch": world * cfg.T, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (expert weights "
+                         f"{cfg.E * 3 * cfg.I * cfg.H * 2 / 1e9:.1f} GB streamed each step)"},
+        "tflops": flops / t_s / 1e12,
+        "layer_roofline": {"frac": layer_frac, "frac_nominal_8tbs_2.25pf": roof_t_nominal / t_s,
+                           "roofline_ms": roof_t * 1e3, "flops": flops, "bytes": bytes_,
+                           "touched_experts": touched, "peak_source": peak_kind},
+        "roofline": roof,
+        "kernels": per_kernel,
+        "cpu_baseline": cpu_base,
+        "clocks": clocks.summary(wall1 - ms / 1e3, wall1),
+        "e2e": {"value": world * cfg.T * args.e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "device_status": status,
+    }
+    print(json.dumps(line), flush=True)
+    if dist:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

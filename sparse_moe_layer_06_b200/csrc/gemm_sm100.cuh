@@ -1,0 +1,475 @@
+// gemm_sm100.cuh -- persistent, warp-specialised grouped GEMM on tcgen05/TMEM.
+//
+// One kernel template serves every contraction of the layer:
+//   EPI_LOGITS      router logits      D[e, tok]  = Wgate[e,:]   . x[tok,:]
+//   EPI_SWIGLU      expert gate/up     G[i, row]  = Wg_e[i,:]    . x_perm[row,:]
+//                                      U[i, row]  = Wu_e[i,:]    . x_perm[row,:]
+//                                      h[row, i]  = silu(clamp(G)) * clamp(U)
+//   EPI_DOWN_ATOMIC expert down+combine y[h, row] = sum_i Wd_e[i,h] * h_perm[row,i]
+//                                      out_acc[token(row), h] += w(row) * y
+//   EPI_DOWN_STORE  expert down        y_perm[row, h] = y
+//
+// The weight matrix is always the MMA "A" operand (M = 128 weight rows per
+// tile) and the token rows are the "B" operand (N = 16..NMAX rows per tile,
+// any multiple of 16).  Putting tokens on N lets one kernel cover a decode
+// batch (a couple of rows per expert: N = 16) and a prefill batch (hundreds of
+// rows per expert: N up to 256) without padding every expert to 128 rows.
+//
+// Roles (192 threads = 6 warps, one CTA per SM, persistent over tiles):
+//   warp 0      TMA producer: fills a STAGES-deep shared-memory ring
+//   warp 1      TMEM owner + MMA issuer (one thread issues tcgen05.mma)
+//   warps 2..5  epilogue: tcgen05.ld the fp32 accumulator, apply the epilogue,
+//               store to global memory; each warp owns one 32-lane TMEM quarter
+// The accumulator is double-buffered in TMEM when it fits, so the epilogue of
+// tile i overlaps the main loop of tile i+1.
+//
+// Operand layouts in shared memory (128-byte swizzle, 1024-byte atoms):
+//   K-major (x, h, gate/up weights): a tile row = 64 bf16 of K = 128 bytes;
+//     8 rows per atom; descriptor SBO = 1024 B; +32 B per K=16 step.
+//   MN-major (down weights, stored [I,H] with H contiguous): each TMA box is
+//     64 K-rows x 64 H-values (128 bytes); two boxes side by side in H make
+//     the 128-wide M tile; descriptor LBO = 8192 B (between the two 64-wide H
+//     halves), SBO = 1024 B (between 8-row K groups); +2048 B per K=16 step.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace moe {
+
+enum EpiKind : int { EPI_LOGITS = 0, EPI_SWIGLU = 1, EPI_DOWN_ATOMIC = 2, EPI_DOWN_STORE = 3 };
+
+enum DeviceError : int { DEV_OK = 0, DEV_ERR_TIMEOUT = 5, DEV_ERR_BAD_INDEX = 6 };
+
+__device__ __forceinline__ void set_device_error(int32_t* status, int code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+// Device-built tile schedule for nseg segments (a segment = the rows that
+// share one weight matrix).  int32 array of 5*(nseg+1) entries:
+//   prefix[nseg+1]  exclusive prefix sum of per-segment chunk counts
+//   b_row0[nseg]    first row of the segment in its B tensor map
+//   out_row0[nseg]  first row of the segment in the output row space
+//   rows[nseg]      rows in the segment
+//   chunk_len[nseg] rows per chunk (multiple of 16, <= NMAX)
+// Tiles are ordered (segment, chunk, weight block) with the weight block
+// fastest, so the CTAs working at the same time share one chunk of token rows
+// and, across neighbouring chunks, the same weight blocks through L2.
+struct SchedPtrs {
+    const int32_t* prefix;
+    const int32_t* b_row0;
+    const int32_t* out_row0;
+    const int32_t* rows;
+    const int32_t* chunk_len;
+};
+
+__host__ __device__ inline SchedPtrs sched_ptrs(const int32_t* base, int nseg) {
+    SchedPtrs p;
+    p.prefix = base;
+    p.b_row0 = base + (nseg + 1);
+    p.out_row0 = base + 2 * (nseg + 1);
+    p.rows = base + 3 * (nseg + 1);
+    p.chunk_len = base + 4 * (nseg + 1);
+    return p;
+}
+
+constexpr int kMaxSegments = 257;  // 256 routed experts + 1 shared expert
+
+struct GemmArgs {
+    CUtensorMap tmA0;  // A (weights) for ordinary segments
+    CUtensorMap tmA1;  // A for the special segment (shared expert)
+    CUtensorMap tmB0;  // B (token rows) for ordinary segments
+    CUtensorMap tmB1;  // B for the special segment
+    const int32_t* sched;  // device schedule, or nullptr for one host-described segment
+    int32_t single_rows;       // sched == nullptr: rows of the only segment
+    int32_t single_chunk_len;  // sched == nullptr: rows per chunk
+    int32_t nseg;
+    int32_t special_seg;   // segment that uses tmA1/tmB1, or -1
+    int32_t K;             // contraction length, multiple of 64
+    int32_t M_total;       // valid A rows per matrix (E, I or H)
+    int32_t a_seg_stride;  // A rows between consecutive segments' matrices in tmA0
+    int32_t a_off0;        // A row offset of the gate (or only) matrix in a segment
+    int32_t a_off1;        // A row offset of the up matrix (EPI_SWIGLU)
+    void* out;
+    int32_t out_ld;
+    int32_t n_tokens;          // EPI_DOWN_ATOMIC: rows of the accumulator
+    const int32_t* row_token;  // EPI_DOWN_ATOMIC: token of each routed row
+    const float* row_weight;   // EPI_DOWN_ATOMIC: routing weight of each routed row
+    int32_t routed_rows;       // rows >= routed_rows belong to the shared expert
+    float clip;                // EPI_SWIGLU clamp limit (+inf: none)
+    int32_t out_f32;           // EPI_DOWN_STORE: fp32 (1) or bf16 (0) output
+    int32_t* status;           // device error word
+};
+
+template <int EPI, int NMAX>
+struct GemmCfg {
+    static_assert(NMAX % 16 == 0 && NMAX >= 16 && NMAX <= 256, "N tile");
+    static constexpr bool kSwiGLU = (EPI == EPI_SWIGLU);
+    static constexpr bool kDown = (EPI == EPI_DOWN_ATOMIC || EPI == EPI_DOWN_STORE);
+    static constexpr int kNumA = kSwiGLU ? 2 : 1;
+    static constexpr int kATileBytes = 128 * 128;  // 128 rows x 64 bf16
+    static constexpr int kABytes = kNumA * kATileBytes;
+    static constexpr int kBBytes = NMAX * 128;  // NMAX rows x 64 bf16
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static_assert(kStageBytes % 1024 == 0, "stage alignment");
+    static constexpr int kAccCols = kSwiGLU ? 2 * NMAX : NMAX;
+    static constexpr int kAccStages = (2 * kAccCols <= 512) ? 2 : 1;
+    static constexpr int kTmemNeed = kAccStages * kAccCols;
+    static constexpr int kTmemCols = kTmemNeed <= 32    ? 32
+                                     : kTmemNeed <= 64  ? 64
+                                     : kTmemNeed <= 128 ? 128
+                                     : kTmemNeed <= 256 ? 256
+                                                        : 512;
+    static constexpr int kRingBudget = 196 * 1024;
+    static constexpr int kStagesRaw = kRingBudget / kStageBytes;
+    static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
+    static_assert(kStages >= 2, "pipeline depth");
+    // ring + 1 KB alignment slack + barriers/flags + the schedule (5 arrays)
+    static constexpr int kBarrierBytes = 256;
+    static constexpr int kSchedBytes = 5 * (kMaxSegments + 1) * 4;
+    static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kBarrierBytes + kSchedBytes;
+    static constexpr int kThreads = 192;
+};
+
+struct TileInfo {
+    int seg, blk, chunk;
+    int b_row, out_row;
+    int n_valid, n_mma;
+    bool special;
+};
+
+// Shared-memory copy of the schedule (same layout as SchedPtrs, nseg+1 stride).
+struct SmemSched {
+    int32_t* prefix;
+    int32_t* b_row0;
+    int32_t* out_row0;
+    int32_t* rows;
+    int32_t* chunk_len;
+};
+
+__device__ __forceinline__ bool decode_tile(int t, int nblk, int nseg, const SmemSched& ss,
+                                            int special_seg, TileInfo& ti) {
+    int lo = 0, hi = nseg;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (ss.prefix[mid] * nblk <= t) lo = mid;
+        else hi = mid;
+    }
+    const int local = t - ss.prefix[lo] * nblk;
+    ti.seg = lo;
+    ti.chunk = local / nblk;
+    ti.blk = local - ti.chunk * nblk;
+    const int cl = ss.chunk_len[lo];
+    const int first = ti.chunk * cl;
+    int n = ss.rows[lo] - first;
+    if (n > cl) n = cl;
+    ti.n_valid = n;
+    ti.n_mma = (n + 15) & ~15;
+    ti.b_row = ss.b_row0[lo] + first;
+    ti.out_row = ss.out_row0[lo] + first;
+    ti.special = (lo == special_seg);
+    return n > 0;
+}
+
+__device__ __forceinline__ float clamp_keep_nan(float v, float lim) {
+    return v > lim ? lim : (v < -lim ? -lim : v);
+}
+
+template <int EPI, int NMAX>
+__global__ void __launch_bounds__(192, 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs args) {
+    using C = GemmCfg<EPI, NMAX>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte aligned ring (the 128-byte swizzle atoms need it)
+    uint8_t* ring = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* tail = ring + C::kStages * C::kStageBytes;
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(tail);
+    uint64_t* empty_bar = full_bar + C::kStages;
+    uint64_t* accf_bar = empty_bar + C::kStages;
+    uint64_t* acce_bar = accf_bar + 2;
+    uint64_t* final_bar = acce_bar + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int32_t* s_sched = reinterpret_cast<int32_t*>(tail + C::kBarrierBytes);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int nseg = args.sched ? args.nseg : 1;
+    SmemSched ss;
+    ss.prefix = s_sched;
+    ss.b_row0 = s_sched + (nseg + 1);
+    ss.out_row0 = s_sched + 2 * (nseg + 1);
+    ss.rows = s_sched + 3 * (nseg + 1);
+    ss.chunk_len = s_sched + 4 * (nseg + 1);
+    if (args.sched) {
+        for (int i = threadIdx.x; i < 5 * (nseg + 1); i += blockDim.x)
+            s_sched[i] = __ldg(args.sched + i);
+    } else if (threadIdx.x == 0) {
+        const int cl = args.single_chunk_len;
+        ss.prefix[0] = 0;
+        ss.prefix[1] = (args.single_rows + cl - 1) / cl;
+        ss.b_row0[0] = 0;
+        ss.out_row0[0] = 0;
+        ss.rows[0] = args.single_rows;
+        ss.chunk_len[0] = cl;
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            ptx::mbar_init(&full_bar[s], 1);
+            ptx::mbar_init(&empty_bar[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            ptx::mbar_init(&accf_bar[a], 1);
+            ptx::mbar_init(&acce_bar[a], 4);
+        }
+        ptx::mbar_init(final_bar, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        ptx::prefetch_tmap(&args.tmA0);
+        ptx::prefetch_tmap(&args.tmA1);
+        ptx::prefetch_tmap(&args.tmB0);
+        ptx::prefetch_tmap(&args.tmB1);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, C::kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int nblk = (args.M_total + 127) / 128;
+    const int total_tiles = ss.prefix[nseg] * nblk;
+    const int ksteps = args.K / 64;
+
+    auto fail = [&](int code) {
+        *abort_flag = 1;
+        set_device_error(args.status, code);
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            const uint64_t pol_w = ptx::policy_evict_first();
+            const uint64_t pol_x = ptx::policy_evict_last();
+            uint32_t stage = 0, phase = 0;
+            uint32_t armed = 0, armed_phase = 0;  // per-stage bits
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
+                TileInfo ti;
+                if (!decode_tile(t, nblk, nseg, ss, args.special_seg, ti)) continue;
+                const CUtensorMap* tA = ti.special ? &args.tmA1 : &args.tmA0;
+                const CUtensorMap* tB = ti.special ? &args.tmB1 : &args.tmB0;
+                const int a_base = ti.special ? 0 : ti.seg * args.a_seg_stride;
+                const uint32_t bytes = C::kABytes + ti.n_mma * 128;
+                for (int kb = 0; kb < ksteps; ++kb) {
+                    if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag)) {
+                        fail(DEV_ERR_TIMEOUT);
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sA = ring + stage * C::kStageBytes;
+                    uint8_t* sB = sA + C::kABytes;
+                    ptx::mbar_arrive_expect_tx(&full_bar[stage], bytes);
+                    armed |= 1u << stage;
+                    armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+                    const int k0 = kb * 64;
+                    if constexpr (C::kDown) {
+                        // MN-major A: two 64(H) x 64(K) boxes side by side in H
+                        const int krow = a_base + args.a_off0 + k0;
+                        ptx::tma_load_2d(sA, tA, ti.blk * 128, krow, &full_bar[stage], pol_w);
+                        ptx::tma_load_2d(sA + 8192, tA, ti.blk * 128 + 64, krow, &full_bar[stage],
+                                         pol_w);
+                    } else {
+                        ptx::tma_load_2d(sA, tA, k0, a_base + args.a_off0 + ti.blk * 128,
+                                         &full_bar[stage], pol_w);
+                        if constexpr (C::kSwiGLU) {
+                            ptx::tma_load_2d(sA + C::kATileBytes, tA, k0,
+                                             a_base + args.a_off1 + ti.blk * 128, &full_bar[stage],
+                                             pol_w);
+                        }
+                    }
+                    for (int q = 0; q < ti.n_mma; q += 16) {
+                        ptx::tma_load_2d(sB + q * 128, tB, k0, ti.b_row + q, &full_bar[stage],
+                                         pol_x);
+                    }
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+            // never leave with bulk copies still writing into this CTA's smem
+            for (int s = 0; s < C::kStages; ++s) {
+                if (armed & (1u << s)) {
+                    ptx::mbar_wait(&full_bar[s], (armed_phase >> s) & 1u, nullptr);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+            bool ok = true;
+            constexpr uint32_t kAMajor = C::kDown ? 1u : 0u;
+            for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
+                TileInfo ti;
+                if (!decode_tile(t, nblk, nseg, ss, args.special_seg, ti)) continue;
+                if (!ptx::mbar_wait(&acce_bar[acc], acc_phase ^ 1, abort_flag)) {
+                    fail(DEV_ERR_TIMEOUT);
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint32_t d0 = tmem_base + acc * C::kAccCols;
+                const uint32_t idesc = ptx::idesc_bf16_f32(128, ti.n_mma, kAMajor, 0);
+                for (int kb = 0; kb < ksteps; ++kb) {
+                    if (!ptx::mbar_wait(&full_bar[stage], phase, abort_flag)) {
+                        fail(DEV_ERR_TIMEOUT);
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t a_addr = ptx::smem_u32(ring + stage * C::kStageBytes);
+                    const uint32_t b_addr = a_addr + C::kABytes;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+                        const uint64_t bdesc = ptx::smem_desc_sw128(b_addr + kk * 32, 16, 1024);
+                        if constexpr (C::kDown) {
+                            const uint64_t adesc =
+                                ptx::smem_desc_sw128(a_addr + kk * 2048, 8192, 1024);
+                            ptx::mma_bf16(d0, adesc, bdesc, idesc, accum);
+                        } else {
+                            const uint64_t adesc = ptx::smem_desc_sw128(a_addr + kk * 32, 16, 1024);
+                            ptx::mma_bf16(d0, adesc, bdesc, idesc, accum);
+                            if constexpr (C::kSwiGLU) {
+                                const uint64_t adesc_u = ptx::smem_desc_sw128(
+                                    a_addr + C::kATileBytes + kk * 32, 16, 1024);
+                                ptx::mma_bf16(d0 + NMAX, adesc_u, bdesc, idesc, accum);
+                            }
+                        }
+                    }
+                    ptx::mma_commit(&empty_bar[stage]);
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (!ok) break;
+                ptx::mma_commit(&accf_bar[acc]);
+                if (++acc == C::kAccStages) {
+                    acc = 0;
+                    acc_phase ^= 1;
+                }
+            }
+            // all issued MMAs must retire before TMEM is released
+            ptx::mma_commit(final_bar);
+            ptx::mbar_wait(final_bar, 0, nullptr);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int quarter = warp & 3;
+        const int row_in_tile = quarter * 32 + lane;
+        uint32_t acc = 0, acc_phase = 0;
+        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+            TileInfo ti;
+            if (!decode_tile(t, nblk, nseg, ss, args.special_seg, ti)) continue;
+            if (!ptx::mbar_wait(&accf_bar[acc], acc_phase, abort_flag)) {
+                fail(DEV_ERR_TIMEOUT);
+                break;
+            }
+            ptx::tc_fence_after();
+            const uint32_t tbase = tmem_base + acc * C::kAccCols +
+                                   (static_cast<uint32_t>(quarter * 32) << 16);
+            const int m = ti.blk * 128 + row_in_tile;
+            const bool m_ok = m < args.M_total;
+            for (int c0 = 0; c0 < ti.n_mma; c0 += 16) {
+                float v[16];
+                ptx::tmem_ld16(tbase + c0, v);
+                if constexpr (EPI == EPI_SWIGLU) {
+                    float u[16];
+                    ptx::tmem_ld16(tbase + NMAX + c0, u);
+                    ptx::tmem_ld_wait();
+                    if (m_ok) {
+                        __nv_bfloat16* hout = reinterpret_cast<__nv_bfloat16*>(args.out);
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            if (c0 + j < ti.n_valid) {
+                                const float g = clamp_keep_nan(v[j], args.clip);
+                                const float uu = clamp_keep_nan(u[j], args.clip);
+                                const float hval = g / (1.0f + __expf(-g)) * uu;
+                                hout[static_cast<size_t>(ti.out_row + c0 + j) * args.out_ld + m] =
+                                    __float2bfloat16_rn(hval);
+                            }
+                        }
+                    }
+                } else if constexpr (EPI == EPI_DOWN_ATOMIC) {
+                    ptx::tmem_ld_wait();
+                    int my_tok = 0;
+                    float my_w = 0.0f;
+                    const int col = c0 + (lane & 15);
+                    if (col < ti.n_valid) {
+                        const int r = ti.out_row + col;
+                        if (r < args.routed_rows) {
+                            my_tok = __ldg(args.row_token + r);
+                            my_w = __ldg(args.row_weight + r);
+                        } else {
+                            my_tok = r - args.routed_rows;
+                            my_w = 1.0f;
+                        }
+                    }
+                    float* oacc = reinterpret_cast<float*>(args.out);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int tok = __shfl_sync(0xffffffffu, my_tok, j);
+                        const float w = __shfl_sync(0xffffffffu, my_w, j);
+                        if (m_ok && c0 + j < ti.n_valid) {
+                            if (static_cast<unsigned>(tok) < static_cast<unsigned>(args.n_tokens)) {
+                                atomicAdd(oacc + static_cast<size_t>(tok) * args.out_ld + m,
+                                          w * v[j]);
+                            } else {
+                                set_device_error(args.status, DEV_ERR_BAD_INDEX);
+                            }
+                        }
+                    }
+                } else {
+                    ptx::tmem_ld_wait();
+                    if (m_ok) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            if (c0 + j < ti.n_valid) {
+                                const size_t o =
+                                    static_cast<size_t>(ti.out_row + c0 + j) * args.out_ld + m;
+                                if (EPI == EPI_LOGITS || args.out_f32) {
+                                    reinterpret_cast<float*>(args.out)[o] = v[j];
+                                } else {
+                                    reinterpret_cast<__nv_bfloat16*>(args.out)[o] =
+                                        __float2bfloat16_rn(v[j]);
+                                }
+                            }
+                        }
+                    }
+                }
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&acce_bar[acc]);
+            if (++acc == C::kAccStages) {
+                acc = 0;
+                acc_phase ^= 1;
+            }
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == 1) ptx::tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+}  // namespace moe

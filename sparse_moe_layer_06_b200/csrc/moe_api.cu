@@ -1,0 +1,820 @@
+// moe_api.cu -- host side of the C ABI declared in include/moe.h:
+// argument validation, workspace carving, TMA tensor-map encoding, kernel
+// launch sequencing, the launch counter and the per-kernel event profiler.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/moe.h"
+#include "gemm_sm100.cuh"
+#include "small_kernels.cuh"
+
+namespace moe {
+namespace {
+
+// ------------------------------------------------------------------ launch bookkeeping
+
+std::atomic<int64_t> g_launches{0};
+
+struct ProfRecord {
+    const char* name;
+    cudaEvent_t start, stop;
+};
+
+struct Profiler {
+    std::mutex mu;
+    bool on = false;
+    std::vector<cudaEvent_t> pool;  // 2 per record
+    std::vector<ProfRecord> recs;
+    size_t cap = 0;
+};
+Profiler g_prof;
+
+struct LaunchScope {
+    cudaEvent_t stop = nullptr;
+    cudaStream_t stream;
+    LaunchScope(const char* name, cudaStream_t s) : stream(s) {
+        if (!g_prof.on) return;
+        std::lock_guard<std::mutex> lk(g_prof.mu);
+        if (!g_prof.on || g_prof.recs.size() >= g_prof.cap) return;
+        ProfRecord r{name, g_prof.pool[2 * g_prof.recs.size()],
+                     g_prof.pool[2 * g_prof.recs.size() + 1]};
+        cudaEventRecord(r.start, s);
+        stop = r.stop;
+        g_prof.recs.push_back(r);
+    }
+    ~LaunchScope() {
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        if (stop) cudaEventRecord(stop, stream);
+    }
+};
+
+#define MOE_LAUNCH(name, stream, ...)              \
+    do {                                           \
+        LaunchScope scope_(name, stream);          \
+        __VA_ARGS__;                               \
+        cudaError_t e_ = cudaGetLastError();       \
+        if (e_ != cudaSuccess) return MOE_ERR_CUDA; \
+    } while (0)
+
+// ------------------------------------------------------------------ device info
+
+int sm_count() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    static int cache[64] = {0};
+    if (dev < 64 && cache[dev]) return cache[dev];
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+    if (dev < 64) cache[dev] = n;
+    return n;
+}
+
+// ------------------------------------------------------------------ tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess) {
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        }
+    });
+    return fn;
+}
+
+// 2D bf16 row-major [rows, cols] tensor, box = 64 columns x box_rows rows,
+// 128-byte swizzle, zero fill outside the tensor.
+bool make_tmap(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || rows <= 0 || cols <= 0) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+    cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ problem checks
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int32_t check_problem(const moe_problem* p) {
+    if (!p) return MOE_ERR_INVALID_ARG;
+    if (p->T < 0) return MOE_ERR_INVALID_ARG;
+    if (p->dtype != MOE_F32 && p->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (p->H < 64 || p->H % 64 != 0 || p->I < 64 || p->I % 64 != 0) return MOE_ERR_UNSUPPORTED;
+    if (p->E < 1 || p->E > kMaxExperts || p->top_k < 1 || p->top_k > p->E)
+        return MOE_ERR_UNSUPPORTED;
+    if (p->num_shared != 0 && p->num_shared != 1) return MOE_ERR_UNSUPPORTED;
+    if (p->T * static_cast<int64_t>(p->top_k + p->num_shared) >= (int64_t(1) << 31))
+        return MOE_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(p->E) * 3 * p->I >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+    if (!std::isfinite(p->routed_scale)) return MOE_ERR_INVALID_ARG;
+    if (std::isnan(p->clip_limit)) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+float effective_clip(const moe_problem* p) {
+    return (p->clip_limit > 0.0f && std::isfinite(p->clip_limit)) ? p->clip_limit : INFINITY;
+}
+
+
+// Token-row tile width for the expert GEMMs, from the mean rows per expert.
+int pick_nmax(double mean_rows) {
+    if (mean_rows >= 96.0) return 256;
+    if (mean_rows >= 48.0) return 128;
+    if (mean_rows >= 12.0) return 64;
+    return 16;
+}
+constexpr int kLogitsNmax = 64;
+
+// ------------------------------------------------------------------ workspace layout
+
+struct Carve {
+    size_t off = 0;
+    size_t take(size_t bytes) {
+        size_t o = off;
+        off += (bytes + 255) & ~size_t(255);
+        return o;
+    }
+};
+
+struct Layout {
+    size_t status, logits, idx, w, hist, base, counts, offsets, sched_gu, sched_dn, pos, src, row_w;
+    size_t x_perm, x_bf16, w_bf16, ws_bf16, h_perm, out_acc, y_bf16, total;
+};
+
+int64_t perm_chunks(int64_t T) { return (T + kPermTokens - 1) / kPermTokens; }
+size_t sched_bytes() { return 5 * (kMaxSegments + 1) * sizeof(int32_t); }
+
+Layout layout_for(const moe_problem* p, int call, int64_t ffn_rows = 0, int ffn_groups = 0) {
+    Layout L{};
+    Carve c;
+    const int64_t T = p->T, H = p->H, E = p->E, I = p->I, k = p->top_k, S = p->num_shared;
+    const bool f32 = p->dtype == MOE_F32;
+    L.status = c.take(256);
+    switch (call) {
+        case MOE_CALL_ROUTER_LOGITS:
+            break;
+        case MOE_CALL_ROUTE:
+            L.logits = c.take(T * E * 4);
+            break;
+        case MOE_CALL_PERMUTE:
+            L.hist = c.take(perm_chunks(T) * E * 4);
+            L.base = c.take(perm_chunks(T) * E * 4);
+            L.counts = c.take(E * 4);
+            break;
+        case MOE_CALL_FFN:
+            L.sched_gu = c.take(sched_bytes());
+            L.sched_dn = c.take(sched_bytes());
+            L.h_perm = c.take(ffn_rows * I * 2);
+            if (f32) {
+                L.x_bf16 = c.take(ffn_rows * H * 2);
+                L.w_bf16 = c.take(static_cast<int64_t>(ffn_groups) * 3 * I * H * 2);
+            }
+            break;
+        case MOE_CALL_COMBINE:
+            break;
+        case MOE_CALL_FORWARD:
+        default:
+            L.logits = c.take(T * E * 4);
+            L.idx = c.take(T * k * 4);
+            L.w = c.take(T * k * 4);
+            L.hist = c.take(perm_chunks(T) * E * 4);
+            L.base = c.take(perm_chunks(T) * E * 4);
+            L.counts = c.take(E * 4);
+            L.offsets = c.take((E + 1) * 4);
+            L.sched_gu = c.take(sched_bytes());
+            L.sched_dn = c.take(sched_bytes());
+            L.pos = c.take(T * k * 4);
+            L.src = c.take(T * k * 4);
+            L.row_w = c.take(T * k * 4);
+            L.x_perm = c.take(T * k * H * 2);
+            L.h_perm = c.take(T * (k + S) * I * 2);
+            L.out_acc = c.take(T * H * 4);
+            if (f32) {
+                L.x_bf16 = c.take(T * H * 2);
+                L.w_bf16 = c.take(E * 3 * I * H * 2);
+                L.ws_bf16 = c.take(S * 3 * I * H * 2);
+            }
+            break;
+    }
+    L.total = c.off;
+    return L;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+    return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+// ------------------------------------------------------------------ GEMM launch
+
+template <int EPI, int NMAX>
+int32_t launch_gemm_n(const GemmArgs& a, int grid, cudaStream_t s, const char* name) {
+    using C = GemmCfg<EPI, NMAX>;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static std::atomic<uint64_t> configured{0};
+    const uint64_t bit = (dev < 64) ? (1ull << dev) : 0;
+    if (!bit || !(configured.load() & bit)) {
+        if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI, NMAX>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::kSmemBytes) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        configured.fetch_or(bit);
+    }
+    MOE_LAUNCH(name, s, grouped_gemm_kernel<EPI, NMAX><<<grid, C::kThreads, C::kSmemBytes, s>>>(a));
+    return MOE_OK;
+}
+
+template <int EPI>
+int32_t launch_gemm(int nmax, const GemmArgs& a, int64_t max_tiles, cudaStream_t s,
+                    const char* name) {
+    int grid = static_cast<int>(std::min<int64_t>(sm_count(), std::max<int64_t>(1, max_tiles)));
+    switch (nmax) {
+        case 16: return launch_gemm_n<EPI, 16>(a, grid, s, name);
+        case 64: return launch_gemm_n<EPI, 64>(a, grid, s, name);
+        case 128: return launch_gemm_n<EPI, 128>(a, grid, s, name);
+        case 256: return launch_gemm_n<EPI, 256>(a, grid, s, name);
+        default: return MOE_ERR_UNSUPPORTED;
+    }
+}
+
+// Upper bound on tiles of a schedule: sum over segments of ceil(rows/nmax)
+// <= rows_total/nmax + nseg, times weight blocks.
+int64_t max_tiles(int64_t rows_total, int nseg, int nmax, int64_t m_total) {
+    return (rows_total / nmax + nseg) * ((m_total + 127) / 128);
+}
+
+GemmArgs base_args(int32_t* status) {
+    GemmArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.special_seg = -1;
+    a.clip = INFINITY;
+    a.status = status;
+    return a;
+}
+
+// Router logits through tcgen05 (bf16 x and gate weight).
+int32_t run_logits_bf16(const moe_problem* p, const void* x, const void* gate_w, float* logits,
+                        int32_t* status, cudaStream_t s) {
+    GemmArgs a = base_args(status);
+    if (!make_tmap(&a.tmA0, gate_w, p->E, p->H, 128)) return MOE_ERR_CUDA;
+    if (!make_tmap(&a.tmB0, x, p->T, p->H, 16)) return MOE_ERR_CUDA;
+    a.tmA1 = a.tmA0;
+    a.tmB1 = a.tmB0;
+    a.sched = nullptr;
+    a.single_rows = static_cast<int32_t>(p->T);
+    a.single_chunk_len = kLogitsNmax;
+    a.nseg = 1;
+    a.K = p->H;
+    a.M_total = p->E;
+    a.out = logits;
+    a.out_ld = p->E;
+    return launch_gemm<EPI_LOGITS>(kLogitsNmax, a, max_tiles(p->T, 1, kLogitsNmax, p->E), s,
+                                   "router_logits_gemm");
+}
+
+int32_t run_logits(const moe_problem* p, const void* x, const void* gate_w, float* logits,
+                   int32_t* status, cudaStream_t s) {
+    if (p->dtype == MOE_BF16) return run_logits_bf16(p, x, gate_w, logits, status, s);
+    MOE_LAUNCH("router_logits_f32", s,
+               router_logits_f32_kernel<<<static_cast<unsigned>(p->T), 256, 0, s>>>(
+                   static_cast<const float*>(x), static_cast<const float*>(gate_w), p->H, p->E,
+                   logits));
+    return MOE_OK;
+}
+
+int32_t run_topk(const moe_problem* p, const float* logits, const float* bias, int32_t* idx,
+                 float* w, cudaStream_t s) {
+    const int warps = 8;
+    const unsigned blocks = static_cast<unsigned>((p->T + warps - 1) / warps);
+    MOE_LAUNCH("route_topk", s,
+               topk_kernel<<<blocks, warps * 32, 0, s>>>(logits, bias, p->T, p->E, p->top_k,
+                                                         p->routed_scale, idx, w));
+    return MOE_OK;
+}
+
+int32_t run_cast(const void* in, void* out, int64_t n, cudaStream_t s) {
+    const int64_t blocks = std::min<int64_t>((n + 255) / 256, 148 * 16);
+    MOE_LAUNCH("cast_f32_bf16", s,
+               cast_f32_bf16_kernel<<<static_cast<unsigned>(std::max<int64_t>(1, blocks)), 256, 0,
+                                      s>>>(static_cast<const float*>(in),
+                                           static_cast<__nv_bfloat16*>(out), n));
+    return MOE_OK;
+}
+
+template <typename TIn, typename TOut>
+int32_t run_gather(const TIn* x, int64_t T, int H, int k, const int32_t* pos, int64_t n_rows,
+                   TOut* x_perm, __nv_bfloat16* x_bf16, float* acc_zero, cudaStream_t s);
+
+}  // namespace
+
+// Copy each token row into its k permuted rows (optionally converting), one
+// warp per token.  Also writes a bf16 copy of x and zeroes the token's fp32
+// accumulator row when asked.
+template <typename TIn, typename TOut>
+__global__ void gather_kernel(const TIn* __restrict__ x, int64_t T, int H, int k,
+                              const int32_t* __restrict__ pos, int64_t n_rows,
+                              TOut* __restrict__ x_perm, __nv_bfloat16* __restrict__ x_bf16,
+                              float* __restrict__ acc_zero) {
+    const int lane = threadIdx.x & 31;
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= T) return;
+    int my_pos = -1;
+    if (lane < k) {
+        my_pos = pos[t * k + lane];
+        if (my_pos < 0 || my_pos >= n_rows) my_pos = -1;
+    }
+    constexpr int kElems = 16 / sizeof(TOut);  // elements per 16-byte output vector
+    const int nvec = H / kElems;
+    for (int v = lane; v < nvec; v += 32) {
+        uint4 packed;
+        uint4 packed_bf16;
+        if constexpr (sizeof(TIn) == sizeof(TOut)) {
+            packed = reinterpret_cast<const uint4*>(x + t * H)[v];
+        } else {
+            // fp32 -> bf16: 8 inputs per output vector
+            const float4 a = reinterpret_cast<const float4*>(x + t * H)[2 * v];
+            const float4 b = reinterpret_cast<const float4*>(x + t * H)[2 * v + 1];
+            __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y);
+            __nv_bfloat162 p1 = __floats2bfloat162_rn(a.z, a.w);
+            __nv_bfloat162 p2 = __floats2bfloat162_rn(b.x, b.y);
+            __nv_bfloat162 p3 = __floats2bfloat162_rn(b.z, b.w);
+            packed.x = *reinterpret_cast<uint32_t*>(&p0);
+            packed.y = *reinterpret_cast<uint32_t*>(&p1);
+            packed.z = *reinterpret_cast<uint32_t*>(&p2);
+            packed.w = *reinterpret_cast<uint32_t*>(&p3);
+            packed_bf16 = packed;
+            if (x_bf16) reinterpret_cast<uint4*>(x_bf16 + t * H)[v] = packed_bf16;
+        }
+        for (int j = 0; j < k; ++j) {
+            const int r = __shfl_sync(0xffffffffu, my_pos, j);
+            if (r >= 0) reinterpret_cast<uint4*>(x_perm + static_cast<int64_t>(r) * H)[v] = packed;
+        }
+    }
+    if (acc_zero) {
+        float4* z = reinterpret_cast<float4*>(acc_zero + t * H);
+        for (int v = lane; v < H / 4; v += 32) z[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
+namespace {
+
+template <typename TIn, typename TOut>
+int32_t run_gather(const TIn* x, int64_t T, int H, int k, const int32_t* pos, int64_t n_rows,
+                   TOut* x_perm, __nv_bfloat16* x_bf16, float* acc_zero, cudaStream_t s) {
+    const int warps = 8;
+    const unsigned blocks = static_cast<unsigned>((T + warps - 1) / warps);
+    MOE_LAUNCH("dispatch_gather", s,
+               gather_kernel<TIn, TOut><<<blocks, warps * 32, 0, s>>>(x, T, H, k, pos, n_rows,
+                                                                      x_perm, x_bf16, acc_zero));
+    return MOE_OK;
+}
+
+// histogram -> scan (+ schedules) -> stable scatter
+int32_t run_dispatch(const moe_problem* p, const int32_t* idx, const float* topk_w, int32_t* hist,
+                     int32_t* base, int32_t* counts, int32_t* offsets, int32_t* sched_gu,
+                     int nmax_gu, int32_t* sched_dn, int nmax_dn, int32_t* pos, int32_t* src,
+                     float* row_w, int32_t* status, cudaStream_t s) {
+    const unsigned nch = static_cast<unsigned>(perm_chunks(p->T));
+    MOE_LAUNCH("dispatch_count", s,
+               dispatch_count_kernel<<<nch, kPermTokens, 0, s>>>(idx, p->T, p->E, p->top_k, hist,
+                                                                 status));
+    MOE_LAUNCH("dispatch_scan", s,
+               dispatch_scan_kernel<<<1, 256, 0, s>>>(hist, static_cast<int>(nch), p->E, p->T,
+                                                      p->top_k, p->num_shared, base, counts,
+                                                      offsets, sched_gu, nmax_gu, sched_dn,
+                                                      nmax_dn));
+    MOE_LAUNCH("dispatch_scatter", s,
+               dispatch_scatter_kernel<<<nch, kPermTokens, 0, s>>>(
+                   idx, topk_w, p->T, p->E, p->top_k, base, offsets, pos, src, row_w, status));
+    return MOE_OK;
+}
+
+template <typename TOut>
+int32_t run_finalize(const float* acc, TOut* out, int64_t n, cudaStream_t s) {
+    const int64_t n4 = n / 4;
+    const int64_t blocks = std::min<int64_t>((n4 + 255) / 256, 148 * 8);
+    MOE_LAUNCH("finalize", s,
+               finalize_kernel<TOut><<<static_cast<unsigned>(std::max<int64_t>(1, blocks)), 256, 0,
+                                       s>>>(acc, out, n4));
+    return MOE_OK;
+}
+
+#define MOE_TRY(expr)                      \
+    do {                                   \
+        int32_t r_ = (expr);               \
+        if (r_ != MOE_OK) return r_;       \
+    } while (0)
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_status_string(int32_t status) {
+    switch (status) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+        case MOE_ERR_CUDA: return "CUDA launch or runtime error";
+        case MOE_ERR_TIMEOUT: return "device wait timed out";
+        case MOE_ERR_BAD_INDEX: return "index input out of range";
+        default: return "unknown status";
+    }
+}
+
+size_t moe_workspace_size(const moe_problem* p, int32_t call) {
+    if (check_problem(p) != MOE_OK) return 0;
+    if (call < MOE_CALL_ROUTE || call > MOE_CALL_FORWARD) return 0;
+    if (call == MOE_CALL_FFN) {
+        // the FFN workspace depends on rows/groups; size it for the routed
+        // rows of this problem (T*top_k) and E groups, the larger of the two
+        // uses (routed experts, or the shared expert over T rows)
+        const int64_t rows = std::max<int64_t>(p->T * p->top_k, p->T);
+        return layout_for(p, call, rows, p->E).total;
+    }
+    return layout_for(p, call).total;
+}
+
+int32_t moe_router_logits(const moe_problem* p, const void* x, const void* gate_w, float* logits,
+                          void* ws, size_t ws_bytes, void* stream) {
+    MOE_TRY(check_problem(p));
+    if (!x || !gate_w || !logits || !ws) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(gate_w) || !aligned16(logits) || !aligned16(ws))
+        return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < layout_for(p, MOE_CALL_ROUTER_LOGITS).total) return MOE_ERR_WORKSPACE;
+    if (p->T == 0) return MOE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return run_logits(p, x, gate_w, logits, at<int32_t>(ws, 0), s);
+}
+
+int32_t moe_route(const moe_problem* p, const void* x, const void* gate_w, const float* bias,
+                  int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes, void* stream) {
+    MOE_TRY(check_problem(p));
+    if (!x || !gate_w || !topk_idx || !topk_w || !ws) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(gate_w) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+    const Layout L = layout_for(p, MOE_CALL_ROUTE);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    if (p->T == 0) return MOE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t* status = at<int32_t>(ws, L.status);
+    float* logits = at<float>(ws, L.logits);
+    MOE_TRY(run_logits(p, x, gate_w, logits, status, s));
+    return run_topk(p, logits, bias, topk_idx, topk_w, s);
+}
+
+int32_t moe_permute(const moe_problem* p, const int32_t* topk_idx, const void* x,
+                    int32_t* offsets, int32_t* pos, int32_t* src_token, void* x_perm, void* ws,
+                    size_t ws_bytes, void* stream) {
+    MOE_TRY(check_problem(p));
+    if (!topk_idx || !x || !offsets || !pos || !src_token || !x_perm || !ws)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(x_perm) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+    const Layout L = layout_for(p, MOE_CALL_PERMUTE);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    if (p->T == 0) {
+        // offsets are all zero for an empty batch
+        if (cudaMemsetAsync(offsets, 0, (p->E + 1) * sizeof(int32_t),
+                            static_cast<cudaStream_t>(stream)) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t* status = at<int32_t>(ws, L.status);
+    MOE_TRY(run_dispatch(p, topk_idx, nullptr, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base),
+                         at<int32_t>(ws, L.counts), offsets, nullptr, 16, nullptr, 16, pos,
+                         src_token, nullptr, status, s));
+    const int64_t n_rows = p->T * p->top_k;
+    if (p->dtype == MOE_BF16) {
+        return run_gather<__nv_bfloat16, __nv_bfloat16>(
+            static_cast<const __nv_bfloat16*>(x), p->T, p->H, p->top_k, pos, n_rows,
+            static_cast<__nv_bfloat16*>(x_perm), nullptr, nullptr, s);
+    }
+    return run_gather<float, float>(static_cast<const float*>(x), p->T, p->H, p->top_k, pos,
+                                    n_rows, static_cast<float*>(x_perm), nullptr, nullptr, s);
+}
+
+int32_t moe_grouped_swiglu_ffn(const moe_problem* p, const void* x_perm, int64_t rows,
+                               const int32_t* offsets, int32_t n_groups, const void* expert_w,
+                               void* y_perm, void* ws, size_t ws_bytes, void* stream) {
+    MOE_TRY(check_problem(p));
+    if (!x_perm || !offsets || !expert_w || !y_perm || !ws) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x_perm) || !aligned16(expert_w) || !aligned16(y_perm) || !aligned16(ws))
+        return MOE_ERR_INVALID_ARG;
+    if (n_groups < 1 || n_groups > kMaxExperts) return MOE_ERR_UNSUPPORTED;
+    if (rows < 0 || rows >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(n_groups) * 3 * p->I >= (int64_t(1) << 31))
+        return MOE_ERR_UNSUPPORTED;
+    const Layout L = layout_for(p, MOE_CALL_FFN, rows, n_groups);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    if (rows == 0) return MOE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t* status = at<int32_t>(ws, L.status);
+    const int64_t H = p->H, I = p->I;
+    const void* xb = x_perm;
+    const void* wb = expert_w;
+    if (p->dtype == MOE_F32) {
+        MOE_TRY(run_cast(x_perm, at<void>(ws, L.x_bf16), rows * H, s));
+        MOE_TRY(run_cast(expert_w, at<void>(ws, L.w_bf16), n_groups * 3 * I * H, s));
+        xb = at<void>(ws, L.x_bf16);
+        wb = at<void>(ws, L.w_bf16);
+    }
+    const int nmax = pick_nmax(static_cast<double>(rows) / n_groups);
+    int32_t* sg = at<int32_t>(ws, L.sched_gu);
+    int32_t* sd = at<int32_t>(ws, L.sched_dn);
+    MOE_LAUNCH("ffn_schedule", s,
+               schedule_from_offsets_kernel<<<1, 32, 0, s>>>(offsets, n_groups, rows, sg, nmax, sd,
+                                                             nmax, status));
+    __nv_bfloat16* h = at<__nv_bfloat16>(ws, L.h_perm);
+    {
+        GemmArgs a = base_args(status);
+        if (!make_tmap(&a.tmA0, wb, static_cast<int64_t>(n_groups) * 3 * I, H, 128))
+            return MOE_ERR_CUDA;
+        if (!make_tmap(&a.tmB0, xb, rows, H, 16)) return MOE_ERR_CUDA;
+        a.tmA1 = a.tmA0;
+        a.tmB1 = a.tmB0;
+        a.sched = sg;
+        a.nseg = n_groups;
+        a.K = static_cast<int32_t>(H);
+        a.M_total = static_cast<int32_t>(I);
+        a.a_seg_stride = static_cast<int32_t>(3 * I);
+        a.a_off0 = 0;
+        a.a_off1 = static_cast<int32_t>(I);
+        a.out = h;
+        a.out_ld = static_cast<int32_t>(I);
+        a.clip = effective_clip(p);
+        MOE_TRY(launch_gemm<EPI_SWIGLU>(nmax, a, max_tiles(rows, n_groups, nmax, I), s,
+                                        "expert_gate_up_gemm"));
+    }
+    {
+        GemmArgs a = base_args(status);
+        if (!make_tmap(&a.tmA0, wb, static_cast<int64_t>(n_groups) * 3 * I, H, 64))
+            return MOE_ERR_CUDA;
+        if (!make_tmap(&a.tmB0, h, rows, I, 16)) return MOE_ERR_CUDA;
+        a.tmA1 = a.tmA0;
+        a.tmB1 = a.tmB0;
+        a.sched = sd;
+        a.nseg = n_groups;
+        a.K = static_cast<int32_t>(I);
+        a.M_total = static_cast<int32_t>(H);
+        a.a_seg_stride = static_cast<int32_t>(3 * I);
+        a.a_off0 = static_cast<int32_t>(2 * I);
+        a.out = y_perm;
+        a.out_ld = static_cast<int32_t>(H);
+        a.out_f32 = p->dtype == MOE_F32 ? 1 : 0;
+        MOE_TRY(launch_gemm<EPI_DOWN_STORE>(nmax, a, max_tiles(rows, n_groups, nmax, H), s,
+                                            "expert_down_gemm"));
+    }
+    return MOE_OK;
+}
+
+int32_t moe_combine(const moe_problem* p, const void* y_perm, const int32_t* pos,
+                    const float* topk_w, const void* shared_y, void* out, void* ws,
+                    size_t ws_bytes, void* stream) {
+    MOE_TRY(check_problem(p));
+    if (!y_perm || !pos || !topk_w || !out || !ws) return MOE_ERR_INVALID_ARG;
+    if (p->num_shared && !shared_y) return MOE_ERR_INVALID_ARG;
+    const Layout L = layout_for(p, MOE_CALL_COMBINE);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    if (p->T == 0) return MOE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t* status = at<int32_t>(ws, L.status);
+    const int64_t n_rows = p->T * p->top_k;
+    const void* sy = p->num_shared ? shared_y : nullptr;
+    const unsigned blocks = static_cast<unsigned>(p->T);
+    if (p->dtype == MOE_BF16) {
+        MOE_LAUNCH("combine", s,
+                   combine_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+                       static_cast<const __nv_bfloat16*>(y_perm), pos, topk_w,
+                       static_cast<const __nv_bfloat16*>(sy), p->T, p->H, p->top_k, n_rows,
+                       static_cast<__nv_bfloat16*>(out), status));
+    } else {
+        MOE_LAUNCH("combine", s,
+                   combine_kernel<float><<<blocks, 256, 0, s>>>(
+                       static_cast<const float*>(y_perm), pos, topk_w,
+                       static_cast<const float*>(sy), p->T, p->H, p->top_k, n_rows,
+                       static_cast<float*>(out), status));
+    }
+    return MOE_OK;
+}
+
+int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, const float* bias,
+                    const void* expert_w, const void* shared_w, void* out, int32_t* idx_out,
+                    float* w_out, void* ws, size_t ws_bytes, void* stream) {
+    MOE_TRY(check_problem(p));
+    if (!x || !gate_w || !expert_w || !out || !ws) return MOE_ERR_INVALID_ARG;
+    if (p->num_shared && !shared_w) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(gate_w) || !aligned16(expert_w) || !aligned16(out) ||
+        !aligned16(ws) || (shared_w && !aligned16(shared_w)))
+        return MOE_ERR_INVALID_ARG;
+    const Layout L = layout_for(p, MOE_CALL_FORWARD);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    if (p->T == 0) return MOE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t* status = at<int32_t>(ws, L.status);
+    const int64_t T = p->T, H = p->H, E = p->E, I = p->I, k = p->top_k, S = p->num_shared;
+    const bool f32 = p->dtype == MOE_F32;
+
+    int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, L.idx);
+    float* w = w_out ? w_out : at<float>(ws, L.w);
+    float* logits = at<float>(ws, L.logits);
+
+    // weights for the tensor-core GEMMs
+    const void* ew = expert_w;
+    const void* sw = shared_w;
+    if (f32) {
+        MOE_TRY(run_cast(expert_w, at<void>(ws, L.w_bf16), E * 3 * I * H, s));
+        ew = at<void>(ws, L.w_bf16);
+        if (S) {
+            MOE_TRY(run_cast(shared_w, at<void>(ws, L.ws_bf16), 3 * I * H, s));
+            sw = at<void>(ws, L.ws_bf16);
+        }
+    }
+
+    // 1. route
+    MOE_TRY(run_logits(p, x, gate_w, logits, status, s));
+    MOE_TRY(run_topk(p, logits, bias, idx, w, s));
+
+    // 2. dispatch bookkeeping + schedules
+    const int nmax = pick_nmax(static_cast<double>(T * k) / E);
+    int32_t* sg = at<int32_t>(ws, L.sched_gu);
+    int32_t* sd = at<int32_t>(ws, L.sched_dn);
+    int32_t* pos = at<int32_t>(ws, L.pos);
+    int32_t* src = at<int32_t>(ws, L.src);
+    float* row_w = at<float>(ws, L.row_w);
+    MOE_TRY(run_dispatch(p, idx, w, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base),
+                         at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets), sg, nmax, sd, nmax,
+                         pos, src, row_w, status, s));
+
+    // 3. gather token rows (x -> x_perm), bf16 copy of x for fp32, zero accumulator
+    __nv_bfloat16* x_perm = at<__nv_bfloat16>(ws, L.x_perm);
+    float* out_acc = at<float>(ws, L.out_acc);
+    const void* x_b = x;
+    if (f32) {
+        MOE_TRY((run_gather<float, __nv_bfloat16>(static_cast<const float*>(x), T, p->H, p->top_k,
+                                                  pos, T * k, x_perm, at<__nv_bfloat16>(ws, L.x_bf16),
+                                                  out_acc, s)));
+        x_b = at<void>(ws, L.x_bf16);
+    } else {
+        MOE_TRY((run_gather<__nv_bfloat16, __nv_bfloat16>(static_cast<const __nv_bfloat16*>(x), T,
+                                                          p->H, p->top_k, pos, T * k, x_perm,
+                                                          nullptr, out_acc, s)));
+    }
+
+    // 4. grouped gate/up GEMM + clamp + SwiGLU (routed experts, then shared)
+    __nv_bfloat16* h = at<__nv_bfloat16>(ws, L.h_perm);
+    const int64_t h_rows = T * (k + S);
+    const int nseg = static_cast<int>(E + S);
+    {
+        GemmArgs a = base_args(status);
+        if (!make_tmap(&a.tmA0, ew, E * 3 * I, H, 128)) return MOE_ERR_CUDA;
+        if (!make_tmap(&a.tmB0, x_perm, T * k, H, 16)) return MOE_ERR_CUDA;
+        if (S) {
+            if (!make_tmap(&a.tmA1, sw, 3 * I, H, 128)) return MOE_ERR_CUDA;
+            if (!make_tmap(&a.tmB1, x_b, T, H, 16)) return MOE_ERR_CUDA;
+        } else {
+            a.tmA1 = a.tmA0;
+            a.tmB1 = a.tmB0;
+        }
+        a.sched = sg;
+        a.nseg = nseg;
+        a.special_seg = S ? static_cast<int32_t>(E) : -1;
+        a.K = static_cast<int32_t>(H);
+        a.M_total = static_cast<int32_t>(I);
+        a.a_seg_stride = static_cast<int32_t>(3 * I);
+        a.a_off0 = 0;
+        a.a_off1 = static_cast<int32_t>(I);
+        a.out = h;
+        a.out_ld = static_cast<int32_t>(I);
+        a.clip = effective_clip(p);
+        MOE_TRY(launch_gemm<EPI_SWIGLU>(nmax, a, max_tiles(h_rows, nseg, nmax, I), s,
+                                        "expert_gate_up_gemm"));
+    }
+    // 5. grouped down GEMM, routing weight + scatter-add into the fp32 accumulator
+    {
+        GemmArgs a = base_args(status);
+        if (!make_tmap(&a.tmA0, ew, E * 3 * I, H, 64)) return MOE_ERR_CUDA;
+        if (!make_tmap(&a.tmB0, h, h_rows, I, 16)) return MOE_ERR_CUDA;
+        if (S) {
+            if (!make_tmap(&a.tmA1, sw, 3 * I, H, 64)) return MOE_ERR_CUDA;
+        } else {
+            a.tmA1 = a.tmA0;
+        }
+        a.tmB1 = a.tmB0;
+        a.sched = sd;
+        a.nseg = nseg;
+        a.special_seg = S ? static_cast<int32_t>(E) : -1;
+        a.K = static_cast<int32_t>(I);
+        a.M_total = static_cast<int32_t>(H);
+        a.a_seg_stride = static_cast<int32_t>(3 * I);
+        a.a_off0 = static_cast<int32_t>(2 * I);
+        a.out = out_acc;
+        a.out_ld = static_cast<int32_t>(H);
+        a.n_tokens = static_cast<int32_t>(T);
+        a.row_token = src;
+        a.row_weight = row_w;
+        a.routed_rows = static_cast<int32_t>(T * k);
+        MOE_TRY(launch_gemm<EPI_DOWN_ATOMIC>(nmax, a, max_tiles(h_rows, nseg, nmax, H), s,
+                                             "expert_down_combine_gemm"));
+    }
+    // 6. output cast
+    if (f32) return run_finalize<float>(out_acc, static_cast<float*>(out), T * H, s);
+    return run_finalize<__nv_bfloat16>(out_acc, static_cast<__nv_bfloat16*>(out), T * H, s);
+}
+
+int32_t moe_read_device_status(const void* ws, int32_t* status_out, void* stream) {
+    if (!ws || !status_out) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(status_out, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+int32_t moe_clear_device_status(void* ws, void* stream) {
+    if (!ws) return MOE_ERR_INVALID_ARG;
+    if (cudaMemsetAsync(ws, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+int64_t moe_launch_count(void) { return g_launches.load(); }
+
+int32_t moe_profile_start(int32_t max_launches) {
+    if (max_launches <= 0) return MOE_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    if (g_prof.on) return MOE_ERR_INVALID_ARG;
+    g_prof.pool.assign(2 * static_cast<size_t>(max_launches), nullptr);
+    for (auto& e : g_prof.pool) {
+        if (cudaEventCreate(&e) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    g_prof.recs.clear();
+    g_prof.cap = static_cast<size_t>(max_launches);
+    g_prof.on = true;
+    return MOE_OK;
+}
+
+int32_t moe_profile_stop(moe_kernel_time* entries, int32_t max_entries, int32_t* n_entries) {
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    if (!g_prof.on) return MOE_ERR_INVALID_ARG;
+    g_prof.on = false;
+    int32_t rc = MOE_OK;
+    int32_t n = 0;
+    for (const ProfRecord& r : g_prof.recs) {
+        if (cudaEventSynchronize(r.stop) != cudaSuccess) {
+            rc = MOE_ERR_CUDA;
+            break;
+        }
+        float ms = 0.0f;
+        if (cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess) {
+            rc = MOE_ERR_CUDA;
+            break;
+        }
+        int32_t i = 0;
+        while (i < n && std::strcmp(entries[i].name, r.name) != 0) ++i;
+        if (i == n) {
+            if (n >= max_entries) continue;
+            entries[n].name = r.name;
+            entries[n].launches = 0;
+            entries[n].total_ms = 0.0;
+            ++n;
+        }
+        entries[i].launches += 1;
+        entries[i].total_ms += ms;
+    }
+    for (auto& e : g_prof.pool)
+        if (e) cudaEventDestroy(e);
+    g_prof.pool.clear();
+    g_prof.recs.clear();
+    if (n_entries) *n_entries = n;
+    return rc;
+}
+
+}  // extern "C"

@@ -1,0 +1,379 @@
+// small_kernels.cuh -- the memory-light steps around the two grouped GEMMs:
+// top-k routing, the fp32 router GEMM, the dispatch bookkeeping (histogram,
+// scan, stable scatter), the row gather, the tile-schedule builder, the
+// deterministic combine, the fp32->bf16 finalize, and dtype casts.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "gemm_sm100.cuh"
+
+namespace moe {
+
+constexpr int kMaxExperts = 256;
+constexpr int kPermTokens = 256;  // tokens per dispatch chunk (one CTA, 8 warps)
+constexpr int kPermWarps = kPermTokens / 32;
+
+// ------------------------------------------------------------------ routing
+
+// Router logits in fp32 for fp32 inputs: logits[t,e] = sum_h x[t,h] * w[e,h].
+// One CTA per token; each warp walks experts, lanes stride over h.
+__global__ void router_logits_f32_kernel(const float* __restrict__ x,
+                                         const float* __restrict__ gate_w, int H, int E,
+                                         float* __restrict__ logits) {
+    const int t = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float* xr = x + static_cast<size_t>(t) * H;
+    for (int e = warp; e < E; e += blockDim.x >> 5) {
+        const float* wr = gate_w + static_cast<size_t>(e) * H;
+        float acc = 0.0f;
+        for (int h = lane; h < H; h += 32) acc = fmaf(xr[h], wr[h], acc);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) logits[static_cast<size_t>(t) * E + e] = acc;
+    }
+}
+
+// Softmax -> top-k -> renormalise -> scale, one warp per token.
+// Selection runs on the fp32 logits (softmax is monotone, so the selected set
+// is the top-k of the probabilities); exact ties go to the lower expert index.
+// The renormalised weights are computed as the softmax over the k selected
+// logits, which equals p_j / sum_sel p (the full-softmax normaliser cancels).
+__global__ void topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
+                            int64_t T, int E, int k, float scale, int32_t* __restrict__ idx_out,
+                            float* __restrict__ w_out) {
+    const int lane = threadIdx.x & 31;
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= T) return;
+    constexpr int kPer = kMaxExperts / 32;
+    float v[kPer];
+    uint32_t taken = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) {
+            float l = logits[t * E + e];
+            if (bias) l += bias[e];
+            v[i] = l;
+        } else {
+            v[i] = 0.0f;
+            taken |= 1u << i;
+        }
+    }
+    float sel_l = 0.0f, top_l = 0.0f;
+    int sel_e = 0;
+    float my_l = 0.0f;
+    int my_e = -1;
+    for (int j = 0; j < k; ++j) {
+        float best = 0.0f;
+        int be = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            if (!(taken & (1u << i))) {
+                const int e = lane + 32 * i;
+                if (be == 0x7fffffff || v[i] > best) {
+                    best = v[i];
+                    be = e;
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            const bool take = (be == 0x7fffffff) ||
+                              (oe != 0x7fffffff && (ob > best || (ob == best && oe < be)));
+            if (take) {
+                best = ob;
+                be = oe;
+            }
+        }
+        sel_l = best;
+        sel_e = be;
+        if ((sel_e & 31) == lane) taken |= 1u << (sel_e >> 5);
+        if (j == 0) top_l = sel_l;
+        if (lane == j) {
+            my_l = sel_l;
+            my_e = sel_e;
+        }
+    }
+    // weights: softmax over the k selected logits (lanes 0..k-1 hold them)
+    const float ex = (lane < k) ? expf(my_l - top_l) : 0.0f;
+    float sum = ex;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane < k) {
+        idx_out[t * k + lane] = my_e;
+        w_out[t * k + lane] = scale * (ex / sum);
+    }
+}
+
+// ------------------------------------------------------------------ dispatch
+
+// Build, for the warp's 32 tokens, one bit mask per expert of the lanes whose
+// token routes to it.  A token's k experts must be distinct; a repeat, or an
+// index outside [0,E), is reported through `status` and skipped.
+__device__ __forceinline__ void build_lane_masks(const int32_t* __restrict__ idx, int64_t T, int E,
+                                                 int k, int64_t t, uint32_t* warp_masks,
+                                                 int32_t* status) {
+    const int lane = threadIdx.x & 31;
+    if (t < T) {
+        for (int j = 0; j < k; ++j) {
+            const int e = idx[t * k + j];
+            if (e < 0 || e >= E) {
+                set_device_error(status, DEV_ERR_BAD_INDEX);
+                continue;
+            }
+            const uint32_t old = atomicOr(&warp_masks[e], 1u << lane);
+            if (old & (1u << lane)) set_device_error(status, DEV_ERR_BAD_INDEX);
+        }
+    }
+}
+
+// Pass 1: per-chunk expert histogram hist[chunk, e].
+__global__ void dispatch_count_kernel(const int32_t* __restrict__ idx, int64_t T, int E, int k,
+                                      int32_t* __restrict__ hist, int32_t* status) {
+    __shared__ uint32_t masks[kPermWarps][kMaxExperts];
+    for (int i = threadIdx.x; i < kPermWarps * kMaxExperts; i += blockDim.x)
+        (&masks[0][0])[i] = 0u;
+    __syncthreads();
+    const int warp = threadIdx.x >> 5;
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * kPermTokens + threadIdx.x;
+    build_lane_masks(idx, T, E, k, t, masks[warp], status);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int c = 0;
+#pragma unroll
+        for (int w = 0; w < kPermWarps; ++w) c += __popc(masks[w][e]);
+        hist[static_cast<size_t>(blockIdx.x) * E + e] = c;
+    }
+}
+
+// Fill a tile schedule (see SchedPtrs) for nseg segments from per-segment
+// row counts; run by one thread.  Segment s covers rows [row0(s), row0(s)+rows(s)).
+__device__ void fill_schedule(int32_t* sched, int nseg, int nmax, const int32_t* seg_rows,
+                              const int32_t* seg_b_row0, const int32_t* seg_out_row0) {
+    const SchedPtrs sp = sched_ptrs(sched, nseg);
+    int32_t* prefix = const_cast<int32_t*>(sp.prefix);
+    int32_t* b_row0 = const_cast<int32_t*>(sp.b_row0);
+    int32_t* out_row0 = const_cast<int32_t*>(sp.out_row0);
+    int32_t* rows = const_cast<int32_t*>(sp.rows);
+    int32_t* chunk_len = const_cast<int32_t*>(sp.chunk_len);
+    int acc = 0;
+    for (int s = 0; s < nseg; ++s) {
+        const int r = seg_rows[s];
+        const int chunks = (r + nmax - 1) / nmax;
+        int cl = 16;
+        if (chunks > 0) {
+            cl = (r + chunks - 1) / chunks;
+            cl = (cl + 15) & ~15;
+        }
+        prefix[s] = acc;
+        b_row0[s] = seg_b_row0[s];
+        out_row0[s] = seg_out_row0[s];
+        rows[s] = r;
+        chunk_len[s] = cl;
+        acc += chunks;
+    }
+    prefix[nseg] = acc;
+}
+
+// Pass 2 (one CTA): per-chunk bases, expert counts and offsets, and the tile
+// schedules of the gate/up and down GEMMs (routed experts, then the shared
+// expert as one more segment when present).
+__global__ void dispatch_scan_kernel(const int32_t* __restrict__ hist, int nchunks, int E,
+                                     int64_t T, int k, int num_shared,
+                                     int32_t* __restrict__ base, int32_t* __restrict__ counts,
+                                     int32_t* __restrict__ offsets, int32_t* sched_gu, int nmax_gu,
+                                     int32_t* sched_dn, int nmax_dn) {
+    __shared__ int32_t s_cnt[kMaxExperts + 1];
+    __shared__ int32_t s_rows[kMaxExperts + 1], s_b0[kMaxExperts + 1], s_o0[kMaxExperts + 1],
+        s_o0b[kMaxExperts + 1];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int running = 0;
+        for (int c = 0; c < nchunks; ++c) {
+            const int v = hist[static_cast<size_t>(c) * E + e];
+            base[static_cast<size_t>(c) * E + e] = running;
+            running += v;
+        }
+        s_cnt[e] = running;
+        counts[e] = running;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int acc = 0;
+        for (int e = 0; e < E; ++e) {
+            offsets[e] = acc;
+            s_rows[e] = s_cnt[e];
+            s_b0[e] = acc;
+            s_o0[e] = acc;
+            s_o0b[e] = acc;
+            acc += s_cnt[e];
+        }
+        offsets[E] = acc;
+        const int routed = static_cast<int>(T * k);
+        int nseg = E;
+        if (num_shared) {
+            s_rows[E] = static_cast<int>(T);
+            s_b0[E] = 0;         // gate/up: the shared expert reads x itself
+            s_o0[E] = routed;    // its h rows follow the routed rows
+            s_o0b[E] = routed;   // down: B rows are those same h rows
+            nseg = E + 1;
+        }
+        if (sched_gu) fill_schedule(sched_gu, nseg, nmax_gu, s_rows, s_b0, s_o0);
+        if (sched_dn) fill_schedule(sched_dn, nseg, nmax_dn, s_rows, s_o0b, s_o0b);
+    }
+}
+
+// Pass 3: stable positions.  Row order inside an expert is (token, slot);
+// a token lists an expert at most once, so ordering by token is enough.
+__global__ void dispatch_scatter_kernel(const int32_t* __restrict__ idx,
+                                        const float* __restrict__ topk_w, int64_t T, int E, int k,
+                                        const int32_t* __restrict__ base,
+                                        const int32_t* __restrict__ offsets,
+                                        int32_t* __restrict__ pos, int32_t* __restrict__ src,
+                                        float* __restrict__ row_w, int32_t* status) {
+    __shared__ uint32_t masks[kPermWarps][kMaxExperts];
+    __shared__ int32_t wbase[kPermWarps][kMaxExperts];
+    for (int i = threadIdx.x; i < kPermWarps * kMaxExperts; i += blockDim.x)
+        (&masks[0][0])[i] = 0u;
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * kPermTokens + threadIdx.x;
+    build_lane_masks(idx, T, E, k, t, masks[warp], nullptr);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int running = offsets[e] + base[static_cast<size_t>(blockIdx.x) * E + e];
+#pragma unroll
+        for (int w = 0; w < kPermWarps; ++w) {
+            wbase[w][e] = running;
+            running += __popc(masks[w][e]);
+        }
+    }
+    __syncthreads();
+    if (t < T) {
+        const uint32_t lt = (1u << lane) - 1u;
+        for (int j = 0; j < k; ++j) {
+            const int e = idx[t * k + j];
+            if (e < 0 || e >= E) continue;
+            const int r = wbase[warp][e] + __popc(masks[warp][e] & lt);
+            pos[t * k + j] = r;
+            src[r] = static_cast<int32_t>(t);
+            if (row_w) row_w[r] = topk_w[t * k + j];
+        }
+    }
+}
+
+// Schedule for a caller-described grouping (staged FFN entry point):
+// segment g covers rows [offsets[g], offsets[g+1]) of x_perm / y_perm.
+__global__ void schedule_from_offsets_kernel(const int32_t* __restrict__ offsets, int ngroups,
+                                             int64_t max_rows, int32_t* sched_gu, int nmax_gu,
+                                             int32_t* sched_dn, int nmax_dn, int32_t* status) {
+    if (threadIdx.x != 0) return;
+    const SchedPtrs sg = sched_ptrs(sched_gu, ngroups);
+    const SchedPtrs sd = sched_ptrs(sched_dn, ngroups);
+    int accg = 0, accd = 0;
+    for (int g = 0; g < ngroups; ++g) {
+        int o0 = offsets[g], o1 = offsets[g + 1];
+        if (o0 < 0 || o1 < o0 || o1 > max_rows) {
+            set_device_error(status, DEV_ERR_BAD_INDEX);
+            o0 = 0;
+            o1 = 0;
+        }
+        const int r = o1 - o0;
+        const int cg = (r + nmax_gu - 1) / nmax_gu;
+        const int cd = (r + nmax_dn - 1) / nmax_dn;
+        int lg = 16, ld = 16;
+        if (cg > 0) lg = (((r + cg - 1) / cg) + 15) & ~15;
+        if (cd > 0) ld = (((r + cd - 1) / cd) + 15) & ~15;
+        const_cast<int32_t*>(sg.prefix)[g] = accg;
+        const_cast<int32_t*>(sg.b_row0)[g] = o0;
+        const_cast<int32_t*>(sg.out_row0)[g] = o0;
+        const_cast<int32_t*>(sg.rows)[g] = r;
+        const_cast<int32_t*>(sg.chunk_len)[g] = lg;
+        const_cast<int32_t*>(sd.prefix)[g] = accd;
+        const_cast<int32_t*>(sd.b_row0)[g] = o0;
+        const_cast<int32_t*>(sd.out_row0)[g] = o0;
+        const_cast<int32_t*>(sd.rows)[g] = r;
+        const_cast<int32_t*>(sd.chunk_len)[g] = ld;
+        accg += cg;
+        accd += cd;
+    }
+    const_cast<int32_t*>(sg.prefix)[ngroups] = accg;
+    const_cast<int32_t*>(sd.prefix)[ngroups] = accd;
+}
+
+// ------------------------------------------------------------------ outputs
+
+// out[t,h] = cast(acc[t,h]), 4 elements per thread.
+template <typename TOut>
+__global__ void finalize_kernel(const float* __restrict__ acc, TOut* __restrict__ out, int64_t n4) {
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const float4 v = reinterpret_cast<const float4*>(acc)[i];
+        if constexpr (sizeof(TOut) == 4) {
+            reinterpret_cast<float4*>(out)[i] = v;
+        } else {
+            __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+            __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+            uint2 p;
+            p.x = *reinterpret_cast<uint32_t*>(&a);
+            p.y = *reinterpret_cast<uint32_t*>(&b);
+            reinterpret_cast<uint2*>(out)[i] = p;
+        }
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T v);
+template <>
+__device__ __forceinline__ float to_f32<float>(float v) {
+    return v;
+}
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {
+    return __bfloat162float(v);
+}
+
+// Deterministic combine: out[t] = sum_j w[t,j] * y_perm[pos[t,j]] (+ shared_y[t]),
+// summed in slot order in fp32.  One CTA per token.
+template <typename T>
+__global__ void combine_kernel(const T* __restrict__ y_perm, const int32_t* __restrict__ pos,
+                               const float* __restrict__ w, const T* __restrict__ shared_y,
+                               int64_t T_, int H, int k, int64_t n_rows, T* __restrict__ out,
+                               int32_t* status) {
+    const int64_t t = blockIdx.x;
+    __shared__ int32_t s_pos[kMaxExperts];
+    __shared__ float s_w[kMaxExperts];
+    for (int j = threadIdx.x; j < k; j += blockDim.x) {
+        int p = pos[t * k + j];
+        if (p < 0 || p >= n_rows) {
+            set_device_error(status, DEV_ERR_BAD_INDEX);
+            p = -1;
+        }
+        s_pos[j] = p;
+        s_w[j] = w[t * k + j];
+    }
+    __syncthreads();
+    for (int h = threadIdx.x; h < H; h += blockDim.x) {
+        float acc = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            if (s_pos[j] >= 0)
+                acc = fmaf(s_w[j], to_f32(y_perm[static_cast<int64_t>(s_pos[j]) * H + h]), acc);
+        }
+        if (shared_y) acc += to_f32(shared_y[t * H + h]);
+        if constexpr (sizeof(T) == 4) out[t * H + h] = acc;
+        else out[t * H + h] = __float2bfloat16_rn(acc);
+    }
+}
+
+__global__ void cast_f32_bf16_kernel(const float* __restrict__ in, __nv_bfloat16* __restrict__ out,
+                                     int64_t n) {
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        out[i] = __float2bfloat16_rn(in[i]);
+    }
+}
+
+}  // namespace moe

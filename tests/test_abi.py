@@ -1,0 +1,137 @@
+"""CPU checks of the C-ABI library: it builds, loads, exports every entry point
+declared in include/moe.h, and its host-side validation rejects bad calls
+before touching the GPU (no CUDA call is made by anything tested here)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from sparse_moe_layer_06_b200 import build, moe
+from sparse_moe_layer_06_b200.workloads import CONFIGS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return moe.load_library()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "moe.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = header_functions()
+    for required in ("moe_route", "moe_permute", "moe_grouped_swiglu_ffn", "moe_combine",
+                     "moe_forward", "moe_workspace_size", "moe_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = header_functions()
+    assert set(names) == set(moe.EXPORTED)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_library_is_sm100a_only_build(lib):
+    # the build flags target exactly sm_100a
+    assert "arch=compute_100a,code=sm_100a" in " ".join(build.NVCC_FLAGS)
+    assert os.path.getsize(build.LIB) > 0
+
+
+def test_status_strings(lib):
+    assert moe.status_string(0) == "ok"
+    assert "workspace" in moe.status_string(3)
+    assert moe.status_string(99) == "unknown status"
+
+
+def problem(**kw):
+    base = dict(T=128, H=256, E=16, I=128, top_k=2, num_shared=1, routed_scale=2.827,
+                clip_limit=10.0, dtype=torch.bfloat16)
+    base.update(kw)
+    return moe.MoEProblem(**base)
+
+
+def test_workspace_sizes_monotone_and_validated(lib):
+    p = problem()
+    sizes = {c: moe.moe_workspace_size(p, c) for c in range(6)}
+    assert all(v >= 256 for v in sizes.values())
+    assert sizes[moe.MOE_CALL_FORWARD] > sizes[moe.MOE_CALL_ROUTE]
+    big = problem(T=4096)
+    assert moe.moe_workspace_size(big, moe.MOE_CALL_FORWARD) > sizes[moe.MOE_CALL_FORWARD]
+    # unsupported shapes report 0
+    for bad in (problem(H=100), problem(I=96), problem(E=300), problem(top_k=17),
+                problem(num_shared=2), problem(T=-1)):
+        assert moe.moe_workspace_size(bad, moe.MOE_CALL_FORWARD) == 0
+    assert moe.moe_workspace_size(p, 42) == 0
+
+
+def test_forward_workspace_covers_the_prefill_buffers(lib):
+    c = CONFIGS["hy4_prefill"]
+    p = moe.MoEProblem.from_config(c)
+    n = moe.moe_workspace_size(p, moe.MOE_CALL_FORWARD)
+    T, H, E, I, k = c.T, c.H, c.E, c.I, c.top_k
+    must = T * k * H * 2 + T * (k + 1) * I * 2 + T * H * 4  # x_perm + h_perm + accumulator
+    assert must <= n < must * 1.1
+
+
+def _call_forward(lib, pc, ws_ptr, ws_bytes, x=1 << 20):
+    P = ctypes.c_void_p
+    return lib.moe_forward(ctypes.byref(pc), P(x), P(x), None, P(x), P(x), P(x), None, None,
+                           P(ws_ptr), ws_bytes, None)
+
+
+def test_host_validation_rejects_before_launch(lib):
+    # fake, never-dereferenced 16-byte-aligned addresses: every call below must
+    # be rejected on the host, before anything reaches the GPU
+    pc = problem().c()
+    ws_need = moe.moe_workspace_size(problem(), moe.MOE_CALL_FORWARD)
+    assert _call_forward(lib, pc, 1 << 24, ws_need - 1) == moe.MOE_ERR_WORKSPACE
+    assert _call_forward(lib, pc, 0, ws_need) == moe.MOE_ERR_INVALID_ARG
+    assert _call_forward(lib, pc, (1 << 24) + 8, ws_need) == moe.MOE_ERR_INVALID_ARG
+    bad = problem(H=100).c()
+    assert _call_forward(lib, bad, 1 << 24, ws_need) == moe.MOE_ERR_UNSUPPORTED
+    nan_scale = problem(routed_scale=float("nan")).c()
+    assert _call_forward(lib, nan_scale, 1 << 24, ws_need) == moe.MOE_ERR_INVALID_ARG
+    # shared expert requested but no weights given
+    P = ctypes.c_void_p
+    x = 1 << 20
+    rc = lib.moe_forward(ctypes.byref(pc), P(x), P(x), None, P(x), None, P(x), None, None,
+                         P(1 << 24), ws_need, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG
+    # an empty batch is a valid no-op that launches nothing
+    before = moe.moe_launch_count()
+    empty = problem(T=0).c()
+    assert _call_forward(lib, empty, 1 << 24, moe.moe_workspace_size(problem(T=0), 5)) == 0
+    assert moe.moe_launch_count() == before
+
+
+def test_ffn_and_permute_validation(lib):
+    pc = problem().c()
+    P = ctypes.c_void_p
+    ws = moe.moe_workspace_size(problem(), moe.MOE_CALL_FFN)
+    x = 1 << 20
+    assert lib.moe_grouped_swiglu_ffn(ctypes.byref(pc), P(x), 64, P(x), 0, P(x), P(x),
+                                      P(1 << 24), ws, None) == moe.MOE_ERR_UNSUPPORTED
+    assert lib.moe_grouped_swiglu_ffn(ctypes.byref(pc), P(x), 64, P(x), 257, P(x), P(x),
+                                      P(1 << 24), ws, None) == moe.MOE_ERR_UNSUPPORTED
+    assert lib.moe_grouped_swiglu_ffn(ctypes.byref(pc), None, 64, P(x), 4, P(x), P(x),
+                                      P(1 << 24), ws, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_permute(ctypes.byref(pc), None, P(x), P(x), P(x), P(x), P(x), P(1 << 24),
+                           1 << 20, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_route(ctypes.byref(pc), P(x), P(x), None, P(x), P(x), P(1 << 24), 0,
+                         None) == moe.MOE_ERR_WORKSPACE
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    p = problem(T=4, H=64, I=64, E=2, top_k=1, num_shared=0)
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        moe.moe_router_logits(p, x, x, torch.zeros(4, 2), torch.zeros(256, dtype=torch.uint8))
