@@ -190,6 +190,35 @@ int32_t moe_forward(const moe_problem* problem, const void* x, const void* gate_
                     void* out, int32_t* topk_idx_out, float* topk_w_out, void* workspace,
                     size_t ws_bytes, void* stream);
 
+/*
+ * moe_route_noalloc -- moe_route for callers that cannot allocate device
+ * memory: no workspace argument, and no allocation of any kind inside.
+ * There is no counterpart on the pages: it is a deployment convenience.
+ * Some callers cannot hand the library a workspace: code that runs while a
+ * CUDA stream is being captured (where cudaMalloc is not allowed), serving
+ * loops whose framework allocator already owns all device memory, and
+ * latency-critical paths that must not call cudaMalloc/cudaFree because those
+ * can synchronise the device.  This entry point keeps its scratch (the fp32
+ * router logits, T*E floats) in a fixed 1 MiB device array built into the
+ * library, which every GPU that loads the library holds until the process
+ * exits.  Arguments and outputs are those of moe_route.
+ *  - Capacity: 256 + 4*T*E bytes must fit in MOE_ROUTE_NOALLOC_SCRATCH_BYTES
+ *    (e.g. T <= 1023 tokens at E = 256); larger problems return
+ *    MOE_ERR_WORKSPACE and enqueue nothing.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - All calls share the one array and it keeps the last call's contents:
+ *    calls that overlap on the GPU (different streams, or different host
+ *    threads, on one device) race and corrupt each other's logits.  Order
+ *    them on one stream.  The device error word in the array is cleared at
+ *    each call and is not reported to the caller.
+ */
+#define MOE_ROUTE_NOALLOC_SCRATCH_BYTES (1u << 20)
+int32_t moe_route_noalloc(const moe_problem* problem, const void* x, const void* gate_w,
+                          const float* logit_bias, int32_t* topk_idx, float* topk_w,
+                          void* stream);
+
 /* Copy the device error word of `workspace` to *status_out (host), waiting
  * for the stream.  Returns MOE_OK or MOE_ERR_CUDA / MOE_ERR_INVALID_ARG. */
 int32_t moe_read_device_status(const void* workspace, int32_t* status_out, void* stream);

@@ -749,6 +749,57 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
     return run_finalize<__nv_bfloat16>(out_acc, static_cast<__nv_bfloat16*>(out), T * H, s);
 }
 
+}  // extern "C"
+
+// ------------------------------------------------------------------ routing without allocation
+//
+// Scratch for moe_route_noalloc: a fixed device array that every GPU which
+// loads this library holds until the process exits.  Bytes [0, 256) hold a
+// device error word (cleared on each call), the rest the fp32 router logits.
+namespace moe {
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;  // 1 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device.  In host code
+// the array's name only stands in for the symbol; the address is looked up
+// once per device (with that device current) and cached.
+void* noalloc_scratch_address() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    static std::mutex mu;
+    static void* addr[64] = {nullptr};
+    std::lock_guard<std::mutex> lk(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return nullptr;
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+int32_t moe_route_noalloc(const moe_problem* p, const void* x, const void* gate_w,
+                          const float* bias, int32_t* topk_idx, float* topk_w, void* stream) {
+    MOE_TRY(check_problem(p));
+    if (!x || !gate_w || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(gate_w)) return MOE_ERR_INVALID_ARG;
+    const size_t need = 256 + static_cast<size_t>(p->T) * p->E * sizeof(float);
+    if (need > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE;
+    if (p->T == 0) return MOE_OK;
+    uint8_t* base = static_cast<uint8_t*>(noalloc_scratch_address());
+    if (!base) return MOE_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t* status = reinterpret_cast<int32_t*>(base);
+    float* logits = reinterpret_cast<float*>(base + 256);
+    if (cudaMemsetAsync(status, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+    MOE_TRY(run_logits(p, x, gate_w, logits, status, s));
+    return run_topk(p, logits, bias, topk_idx, topk_w, s);
+}
+
 int32_t moe_read_device_status(const void* ws, int32_t* status_out, void* stream) {
     if (!ws || !status_out) return MOE_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

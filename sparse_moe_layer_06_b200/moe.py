@@ -31,7 +31,9 @@ EXPORTED = (
     "moe_workspace_size", "moe_status_string", "moe_router_logits", "moe_route", "moe_permute",
     "moe_grouped_swiglu_ffn", "moe_combine", "moe_forward", "moe_read_device_status",
     "moe_clear_device_status", "moe_launch_count", "moe_profile_start", "moe_profile_stop",
+    "moe_route_noalloc",
 )
+ROUTE_NOALLOC_SCRATCH_BYTES = 1 << 20
 
 
 class MoEProblemC(ctypes.Structure):
@@ -109,6 +111,7 @@ def load_library(path: str = LIB_PATH):
             "moe_launch_count": (I64, []),
             "moe_profile_start": (I32, [I32]),
             "moe_profile_stop": (I32, [ctypes.POINTER(KernelTimeC), I32, ctypes.POINTER(I32)]),
+            "moe_route_noalloc": (I32, [PP, P, P, P, P, P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -177,6 +180,20 @@ def moe_route(problem, x, gate_w, logit_bias, topk_idx, topk_w, workspace, strea
         _ptr(logit_bias, torch.float32, "logit_bias", optional=True),
         _ptr(topk_idx, torch.int32, "topk_idx"), _ptr(topk_w, torch.float32, "topk_w"),
         _ptr(workspace, None, "workspace"), workspace.numel(), _stream(stream)), "moe_route")
+
+
+def moe_route_noalloc(problem, x, gate_w, logit_bias, topk_idx, topk_w, stream=None):
+    """moe_route without a workspace: for callers that cannot allocate device
+    memory (stream capture in progress, a framework allocator owning all
+    memory, hot paths that must not synchronise).  Scratch is a fixed 1 MiB
+    device array inside the library; T*E*4 + 256 bytes must fit in it.
+    Calls that overlap on the GPU race on that array."""
+    pc = problem.c()
+    _check(load_library().moe_route_noalloc(
+        ctypes.byref(pc), _ptr(x, problem.dtype, "x"), _ptr(gate_w, problem.dtype, "gate_w"),
+        _ptr(logit_bias, torch.float32, "logit_bias", optional=True),
+        _ptr(topk_idx, torch.int32, "topk_idx"), _ptr(topk_w, torch.float32, "topk_w"),
+        _stream(stream)), "moe_route_noalloc")
 
 
 def moe_permute(problem, topk_idx, x, offsets, pos, src_token, x_perm, workspace, stream=None):
