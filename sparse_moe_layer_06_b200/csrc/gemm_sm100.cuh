@@ -77,11 +77,19 @@ __host__ __device__ inline SchedPtrs sched_ptrs(const int32_t* base, int nseg) {
 
 constexpr int kMaxSegments = 257;  // 256 routed experts + 1 shared expert
 
+// Token rows are fetched with TMA boxes of 16 << j rows (j = 0..4): a tile of
+// n rows (a multiple of 16) takes one box per set bit of n/16, so a typical
+// prefill tile needs one or two bulk copies per pipeline stage instead of n/16.
+constexpr int kNumBoxSizes = 5;
+
 struct GemmArgs {
-    CUtensorMap tmA0;  // A (weights) for ordinary segments
-    CUtensorMap tmA1;  // A for the special segment (shared expert)
-    CUtensorMap tmB0;  // B (token rows) for ordinary segments
-    CUtensorMap tmB1;  // B for the special segment
+    // A (weights).  EPI_SWIGLU: 3D map {H, I, matrices} with a {64, 128, 2} box
+    // (gate and up tiles of one expert in one copy); EPI_DOWN_*: 2D map over
+    // the [rows, H] view with a {64, 64} box; EPI_LOGITS: 2D {64, 128*MB}.
+    CUtensorMap tmA0;                // ordinary segments
+    CUtensorMap tmA1;                // the special segment (shared expert)
+    CUtensorMap tmB0[kNumBoxSizes];  // B (token rows), box {64, 16 << j}
+    CUtensorMap tmB1[kNumBoxSizes];  // B for the special segment
     const int32_t* sched;  // device schedule, or nullptr for one host-described segment
     int32_t single_rows;       // sched == nullptr: rows of the only segment
     int32_t single_chunk_len;  // sched == nullptr: rows per chunk
@@ -89,9 +97,9 @@ struct GemmArgs {
     int32_t special_seg;   // segment that uses tmA1/tmB1, or -1
     int32_t K;             // contraction length, multiple of 64
     int32_t M_total;       // valid A rows per matrix (E, I or H)
-    int32_t a_seg_stride;  // A rows between consecutive segments' matrices in tmA0
-    int32_t a_off0;        // A row offset of the gate (or only) matrix in a segment
-    int32_t a_off1;        // A row offset of the up matrix (EPI_SWIGLU)
+    int32_t a_seg_stride;  // A rows (EPI_SWIGLU: matrices) between segments in tmA0
+    int32_t a_off0;        // A row (EPI_SWIGLU: matrix) offset of the first matrix
+    int32_t a_off1;        // unused (kept zero)
     void* out;
     int32_t out_ld;
     int32_t n_tokens;          // EPI_DOWN_ATOMIC: rows of the accumulator
@@ -100,21 +108,30 @@ struct GemmArgs {
     int32_t routed_rows;       // rows >= routed_rows belong to the shared expert
     float clip;                // EPI_SWIGLU clamp limit (+inf: none)
     int32_t out_f32;           // EPI_DOWN_STORE: fp32 (1) or bf16 (0) output
+    int32_t l2_hints;          // 1: weights evict-first, token rows evict-last; 0: none
     int32_t* status;           // device error word
 };
 
-template <int EPI, int NMAX>
+// Compile-time shape of one instantiation.
+//   NMAX  largest token-row tile (MMA N), a multiple of 16 in [16, 256]
+//   MB    128-row weight sub-tiles per tile: the gate and the up matrix for
+//         EPI_SWIGLU (MB = 2), else 1 or 2 adjacent 128-row blocks of one
+//         matrix (two MMAs sharing each token tile)
+// The pipeline depth is whatever fits the 227 KB of shared memory.
+template <int EPI, int NMAX, int MB>
 struct GemmCfg {
     static_assert(NMAX % 16 == 0 && NMAX >= 16 && NMAX <= 256, "N tile");
+    static_assert(MB == 1 || MB == 2, "weight sub-tiles");
+    static_assert(EPI != EPI_SWIGLU || MB == 2, "gate/up needs both matrices");
     static constexpr bool kSwiGLU = (EPI == EPI_SWIGLU);
     static constexpr bool kDown = (EPI == EPI_DOWN_ATOMIC || EPI == EPI_DOWN_STORE);
-    static constexpr int kNumA = kSwiGLU ? 2 : 1;
+    static constexpr int kNumA = MB;
     static constexpr int kATileBytes = 128 * 128;  // 128 rows x 64 bf16
     static constexpr int kABytes = kNumA * kATileBytes;
     static constexpr int kBBytes = NMAX * 128;  // NMAX rows x 64 bf16
     static constexpr int kStageBytes = kABytes + kBBytes;
     static_assert(kStageBytes % 1024 == 0, "stage alignment");
-    static constexpr int kAccCols = kSwiGLU ? 2 * NMAX : NMAX;
+    static constexpr int kAccCols = kNumA * NMAX;  // sub-tile j at column j*NMAX
     static constexpr int kAccStages = (2 * kAccCols <= 512) ? 2 : 1;
     static constexpr int kTmemNeed = kAccStages * kAccCols;
     static constexpr int kTmemCols = kTmemNeed <= 32    ? 32
@@ -122,14 +139,18 @@ struct GemmCfg {
                                      : kTmemNeed <= 128 ? 128
                                      : kTmemNeed <= 256 ? 256
                                                         : 512;
-    static constexpr int kRingBudget = 196 * 1024;
-    static constexpr int kStagesRaw = kRingBudget / kStageBytes;
+    static_assert(kTmemNeed <= 512, "TMEM columns");
+    // tail: 1 KB alignment slack + barriers/flags + the schedule (5 arrays)
+    // + (EPI_DOWN_ATOMIC) two buffers of the token and weight of each column
+    static constexpr int kBarrierBytes = 512;
+    static constexpr int kSchedBytes = 5 * (kMaxSegments + 1) * 4;
+    static constexpr int kMetaBytes = (EPI == EPI_DOWN_ATOMIC) ? 2 * NMAX * 8 : 0;
+    static constexpr int kTailBytes = 1024 + kBarrierBytes + kSchedBytes + kMetaBytes;
+    static constexpr int kMaxSmem = 227 * 1024;
+    static constexpr int kStagesRaw = (kMaxSmem - kTailBytes) / kStageBytes;
     static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
     static_assert(kStages >= 2, "pipeline depth");
-    // ring + 1 KB alignment slack + barriers/flags + the schedule (5 arrays)
-    static constexpr int kBarrierBytes = 256;
-    static constexpr int kSchedBytes = 5 * (kMaxSegments + 1) * 4;
-    static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kBarrierBytes + kSchedBytes;
+    static constexpr int kSmemBytes = kStages * kStageBytes + kTailBytes;
     static constexpr int kThreads = 192;
 };
 
@@ -177,9 +198,9 @@ __device__ __forceinline__ float clamp_keep_nan(float v, float lim) {
     return v > lim ? lim : (v < -lim ? -lim : v);
 }
 
-template <int EPI, int NMAX>
+template <int EPI, int NMAX, int MB>
 __global__ void __launch_bounds__(192, 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs args) {
-    using C = GemmCfg<EPI, NMAX>;
+    using C = GemmCfg<EPI, NMAX, MB>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned ring (the 128-byte swizzle atoms need it)
     uint8_t* ring = reinterpret_cast<uint8_t*>(
@@ -190,9 +211,11 @@ __global__ void __launch_bounds__(192, 1) grouped_gemm_kernel(const __grid_const
     uint64_t* accf_bar = empty_bar + C::kStages;
     uint64_t* acce_bar = accf_bar + 2;
     uint64_t* final_bar = acce_bar + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
+    uint64_t* metaf_bar = final_bar + 1;  // EPI_DOWN_ATOMIC column metadata ready (x2)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(metaf_bar + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int32_t* s_sched = reinterpret_cast<int32_t*>(tail + C::kBarrierBytes);
+    uint8_t* s_meta = tail + C::kBarrierBytes + C::kSchedBytes;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -225,14 +248,17 @@ __global__ void __launch_bounds__(192, 1) grouped_gemm_kernel(const __grid_const
             ptx::mbar_init(&acce_bar[a], 4);
         }
         ptx::mbar_init(final_bar, 1);
+        ptx::mbar_init(&metaf_bar[0], 4);
+        ptx::mbar_init(&metaf_bar[1], 4);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
-    if (warp == 0 && lane == 0) {
-        ptx::prefetch_tmap(&args.tmA0);
-        ptx::prefetch_tmap(&args.tmA1);
-        ptx::prefetch_tmap(&args.tmB0);
-        ptx::prefetch_tmap(&args.tmB1);
+    if (warp == 0 && lane < 2 + 2 * kNumBoxSizes) {
+        const CUtensorMap* m = lane == 0   ? &args.tmA0
+                               : lane == 1 ? &args.tmA1
+                               : lane < 2 + kNumBoxSizes ? &args.tmB0[lane - 2]
+                                                         : &args.tmB1[lane - 2 - kNumBoxSizes];
+        ptx::prefetch_tmap(m);
     }
     if (warp == 1) {
         ptx::tmem_alloc(tmem_slot, C::kTmemCols);
@@ -243,7 +269,10 @@ __global__ void __launch_bounds__(192, 1) grouped_gemm_kernel(const __grid_const
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    const int nblk = (args.M_total + 127) / 128;
+    // a tile covers 128 weight rows per sub-tile; gate/up sub-tiles are the two
+    // matrices at the same rows, other sub-tiles are adjacent row blocks
+    constexpr int kRowsPerTile = C::kSwiGLU ? 128 : 128 * MB;
+    const int nblk = (args.M_total + kRowsPerTile - 1) / kRowsPerTile;
     const int total_tiles = ss.prefix[nseg] * nblk;
     const int ksteps = args.K / 64;
 
@@ -255,8 +284,10 @@ __global__ void __launch_bounds__(192, 1) grouped_gemm_kernel(const __grid_const
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            const uint64_t pol_w = ptx::policy_evict_first();
-            const uint64_t pol_x = ptx::policy_evict_last();
+            const uint64_t pol_w =
+                args.l2_hints ? ptx::policy_evict_first() : ptx::policy_evict_normal();
+            const uint64_t pol_x =
+                args.l2_hints ? ptx::policy_evict_last() : ptx::policy_evict_normal();
             uint32_t stage = 0, phase = 0;
             uint32_t armed = 0, armed_phase = 0;  // per-stage bits
             bool ok = true;
@@ -264,7 +295,7 @@ __global__ void __launch_bounds__(192, 1) grouped_gemm_kernel(const __grid_const
                 TileInfo ti;
                 if (!decode_tile(t, nblk, nseg, ss, args.special_seg, ti)) continue;
                 const CUtensorMap* tA = ti.special ? &args.tmA1 : &args.tmA0;
-                const CUtensorMap* tB = ti.special ? &args.tmB1 : &args.tmB0;
+                const CUtensorMap* tB = ti.special ? args.tmB1 : args.tmB0;
                 const int a_base = ti.special ? 0 : ti.seg * args.a_seg_stride;
                 const uint32_t bytes = C::kABytes + ti.n_mma * 128;
                 for (int kb = 0; kb < ksteps; ++kb) {
@@ -280,23 +311,43 @@ __global__ void __launch_bounds__(192, 1) grouped_gemm_kernel(const __grid_const
                     armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
                     const int k0 = kb * 64;
                     if constexpr (C::kDown) {
-                        // MN-major A: two 64(H) x 64(K) boxes side by side in H
+                        // MN-major A: per sub-tile two 64(H) x 64(K) boxes side
+                        // by side in H
                         const int krow = a_base + args.a_off0 + k0;
-                        ptx::tma_load_2d(sA, tA, ti.blk * 128, krow, &full_bar[stage], pol_w);
-                        ptx::tma_load_2d(sA + 8192, tA, ti.blk * 128 + 64, krow, &full_bar[stage],
-                                         pol_w);
-                    } else {
-                        ptx::tma_load_2d(sA, tA, k0, a_base + args.a_off0 + ti.blk * 128,
+#pragma unroll
+                        for (int j = 0; j < MB; ++j) {
+                            const int h0 = (ti.blk * MB + j) * 128;
+                            ptx::tma_load_2d(sA + j * C::kATileBytes, tA, h0, krow,
+                                             &full_bar[stage], pol_w);
+                            ptx::tma_load_2d(sA + j * C::kATileBytes + 8192, tA, h0 + 64, krow,
+                                             &full_bar[stage], pol_w);
+                        }
+                    } else if constexpr (C::kSwiGLU) {
+                        // gate and up tiles (adjacent matrices) in one 3D copy
+                        ptx::tma_load_3d(sA, tA, k0, ti.blk * 128, a_base + args.a_off0,
                                          &full_bar[stage], pol_w);
-                        if constexpr (C::kSwiGLU) {
-                            ptx::tma_load_2d(sA + C::kATileBytes, tA, k0,
-                                             a_base + args.a_off1 + ti.blk * 128, &full_bar[stage],
-                                             pol_w);
+                    } else if constexpr (MB == 2) {
+                        // both 128-row blocks in one 256-row box
+                        ptx::tma_load_2d(sA, tA, k0, a_base + args.a_off0 + ti.blk * 256,
+                                         &full_bar[stage], pol_w);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < MB; ++j) {
+                            ptx::tma_load_2d(sA + j * C::kATileBytes, tA, k0,
+                                             a_base + args.a_off0 + (ti.blk * MB + j) * 128,
+                                             &full_bar[stage], pol_w);
                         }
                     }
-                    for (int q = 0; q < ti.n_mma; q += 16) {
-                        ptx::tma_load_2d(sB + q * 128, tB, k0, ti.b_row + q, &full_bar[stage],
-                                         pol_x);
+                    {
+                        int q = 0;
+#pragma unroll
+                        for (int j = kNumBoxSizes - 1; j >= 0; --j) {
+                            if ((ti.n_mma >> 4) & (1 << j)) {
+                                ptx::tma_load_2d(sB + q * 128, &tB[j], k0, ti.b_row + q,
+                                                 &full_bar[stage], pol_x);
+                                q += 16 << j;
+                            }
+                        }
                     }
                     if (++stage == C::kStages) {
                         stage = 0;
@@ -340,18 +391,13 @@ __global__ void __launch_bounds__(192, 1) grouped_gemm_kernel(const __grid_const
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
                         const uint64_t bdesc = ptx::smem_desc_sw128(b_addr + kk * 32, 16, 1024);
-                        if constexpr (C::kDown) {
+#pragma unroll
+                        for (int j = 0; j < MB; ++j) {
+                            const uint32_t a_sub = a_addr + j * C::kATileBytes;
                             const uint64_t adesc =
-                                ptx::smem_desc_sw128(a_addr + kk * 2048, 8192, 1024);
-                            ptx::mma_bf16(d0, adesc, bdesc, idesc, accum);
-                        } else {
-                            const uint64_t adesc = ptx::smem_desc_sw128(a_addr + kk * 32, 16, 1024);
-                            ptx::mma_bf16(d0, adesc, bdesc, idesc, accum);
-                            if constexpr (C::kSwiGLU) {
-                                const uint64_t adesc_u = ptx::smem_desc_sw128(
-                                    a_addr + C::kATileBytes + kk * 32, 16, 1024);
-                                ptx::mma_bf16(d0 + NMAX, adesc_u, bdesc, idesc, accum);
-                            }
+                                C::kDown ? ptx::smem_desc_sw128(a_sub + kk * 2048, 8192, 1024)
+                                         : ptx::smem_desc_sw128(a_sub + kk * 32, 16, 1024);
+                            ptx::mma_bf16(d0 + j * NMAX, adesc, bdesc, idesc, accum);
                         }
                     }
                     ptx::mma_commit(&empty_bar[stage]);
@@ -376,9 +422,42 @@ __global__ void __launch_bounds__(192, 1) grouped_gemm_kernel(const __grid_const
         const int quarter = warp & 3;
         const int row_in_tile = quarter * 32 + lane;
         uint32_t acc = 0, acc_phase = 0;
+        uint32_t mi = 0, meta_phase = 0;
         for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
             TileInfo ti;
             if (!decode_tile(t, nblk, nseg, ss, args.special_seg, ti)) continue;
+            int32_t* w_tok = reinterpret_cast<int32_t*>(s_meta) + mi * 2 * NMAX;
+            float* w_wt = reinterpret_cast<float*>(w_tok + NMAX);
+            if constexpr (EPI == EPI_DOWN_ATOMIC) {
+                // token and routing weight of every column, fetched by the four
+                // epilogue warps together (a quarter each) before the
+                // accumulator is ready, so the loads overlap the main loop.
+                // Two buffers alternate by tile; a warp only refills a buffer
+                // after all four have published the next tile's quarter, i.e.
+                // after all of them finished reading it.
+                for (int c = (warp - 2) * 32 + lane; c < ti.n_valid; c += 128) {
+                    const int r = ti.out_row + c;
+                    int tok;
+                    float wt;
+                    if (r < args.routed_rows) {
+                        tok = __ldg(args.row_token + r);
+                        wt = __ldg(args.row_weight + r);
+                    } else {
+                        tok = r - args.routed_rows;
+                        wt = 1.0f;
+                    }
+                    w_tok[c] = tok;
+                    w_wt[c] = wt;
+                }
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&metaf_bar[mi]);
+                if (!ptx::mbar_wait(&metaf_bar[mi], meta_phase, abort_flag)) {
+                    fail(DEV_ERR_TIMEOUT);
+                    break;
+                }
+                mi ^= 1;
+                if (mi == 0) meta_phase ^= 1;
+            }
             if (!ptx::mbar_wait(&accf_bar[acc], acc_phase, abort_flag)) {
                 fail(DEV_ERR_TIMEOUT);
                 break;
@@ -386,70 +465,65 @@ __global__ void __launch_bounds__(192, 1) grouped_gemm_kernel(const __grid_const
             ptx::tc_fence_after();
             const uint32_t tbase = tmem_base + acc * C::kAccCols +
                                    (static_cast<uint32_t>(quarter * 32) << 16);
-            const int m = ti.blk * 128 + row_in_tile;
-            const bool m_ok = m < args.M_total;
-            for (int c0 = 0; c0 < ti.n_mma; c0 += 16) {
-                float v[16];
-                ptx::tmem_ld16(tbase + c0, v);
-                if constexpr (EPI == EPI_SWIGLU) {
-                    float u[16];
+            if constexpr (C::kSwiGLU) {
+                const int m = ti.blk * 128 + row_in_tile;
+                const bool m_ok = m < args.M_total;
+                __nv_bfloat16* hout = reinterpret_cast<__nv_bfloat16*>(args.out);
+                for (int c0 = 0; c0 < ti.n_mma; c0 += 16) {
+                    float g[16], u[16];
+                    ptx::tmem_ld16(tbase + c0, g);
                     ptx::tmem_ld16(tbase + NMAX + c0, u);
                     ptx::tmem_ld_wait();
                     if (m_ok) {
-                        __nv_bfloat16* hout = reinterpret_cast<__nv_bfloat16*>(args.out);
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             if (c0 + j < ti.n_valid) {
-                                const float g = clamp_keep_nan(v[j], args.clip);
+                                const float gg = clamp_keep_nan(g[j], args.clip);
                                 const float uu = clamp_keep_nan(u[j], args.clip);
-                                const float hval = g / (1.0f + __expf(-g)) * uu;
+                                const float hval = gg / (1.0f + __expf(-gg)) * uu;
                                 hout[static_cast<size_t>(ti.out_row + c0 + j) * args.out_ld + m] =
                                     __float2bfloat16_rn(hval);
                             }
                         }
                     }
-                } else if constexpr (EPI == EPI_DOWN_ATOMIC) {
-                    ptx::tmem_ld_wait();
-                    int my_tok = 0;
-                    float my_w = 0.0f;
-                    const int col = c0 + (lane & 15);
-                    if (col < ti.n_valid) {
-                        const int r = ti.out_row + col;
-                        if (r < args.routed_rows) {
-                            my_tok = __ldg(args.row_token + r);
-                            my_w = __ldg(args.row_weight + r);
-                        } else {
-                            my_tok = r - args.routed_rows;
-                            my_w = 1.0f;
-                        }
-                    }
-                    float* oacc = reinterpret_cast<float*>(args.out);
+                }
+            } else {
+#pragma unroll 1
+                for (int sub = 0; sub < MB; ++sub) {
+                    const int m = (ti.blk * MB + sub) * 128 + row_in_tile;
+                    const bool m_ok = m < args.M_total;
+                    for (int c0 = 0; c0 < ti.n_mma; c0 += 16) {
+                        float v[16];
+                        ptx::tmem_ld16(tbase + sub * NMAX + c0, v);
+                        ptx::tmem_ld_wait();
+                        if constexpr (EPI == EPI_DOWN_ATOMIC) {
+                            float* oacc = reinterpret_cast<float*>(args.out);
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int tok = __shfl_sync(0xffffffffu, my_tok, j);
-                        const float w = __shfl_sync(0xffffffffu, my_w, j);
-                        if (m_ok && c0 + j < ti.n_valid) {
-                            if (static_cast<unsigned>(tok) < static_cast<unsigned>(args.n_tokens)) {
-                                atomicAdd(oacc + static_cast<size_t>(tok) * args.out_ld + m,
-                                          w * v[j]);
-                            } else {
-                                set_device_error(args.status, DEV_ERR_BAD_INDEX);
+                            for (int j = 0; j < 16; ++j) {
+                                const int c = c0 + j;
+                                if (m_ok && c < ti.n_valid) {
+                                    const int tok = w_tok[c];
+                                    if (static_cast<unsigned>(tok) <
+                                        static_cast<unsigned>(args.n_tokens)) {
+                                        atomicAdd(oacc + static_cast<size_t>(tok) * args.out_ld + m,
+                                                  w_wt[c] * v[j]);
+                                    } else {
+                                        set_device_error(args.status, DEV_ERR_BAD_INDEX);
+                                    }
+                                }
                             }
-                        }
-                    }
-                } else {
-                    ptx::tmem_ld_wait();
-                    if (m_ok) {
+                        } else if (m_ok) {
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            if (c0 + j < ti.n_valid) {
-                                const size_t o =
-                                    static_cast<size_t>(ti.out_row + c0 + j) * args.out_ld + m;
-                                if (EPI == EPI_LOGITS || args.out_f32) {
-                                    reinterpret_cast<float*>(args.out)[o] = v[j];
-                                } else {
-                                    reinterpret_cast<__nv_bfloat16*>(args.out)[o] =
-                                        __float2bfloat16_rn(v[j]);
+                            for (int j = 0; j < 16; ++j) {
+                                if (c0 + j < ti.n_valid) {
+                                    const size_t o =
+                                        static_cast<size_t>(ti.out_row + c0 + j) * args.out_ld + m;
+                                    if (EPI == EPI_LOGITS || args.out_f32) {
+                                        reinterpret_cast<float*>(args.out)[o] = v[j];
+                                    } else {
+                                        reinterpret_cast<__nv_bfloat16*>(args.out)[o] =
+                                            __float2bfloat16_rn(v[j]);
+                                    }
                                 }
                             }
                         }

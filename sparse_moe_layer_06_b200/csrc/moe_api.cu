@@ -8,6 +8,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -115,6 +116,29 @@ bool make_tmap(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int 
     return r == CUDA_SUCCESS;
 }
 
+// Gate/up weights as a 3D bf16 tensor {H, I, n_mats} (n_mats [I,H] matrices
+// back to back), box {64, 128, 2}: one copy brings the gate and the up tile.
+bool make_tmap_gateup(CUtensorMap* m, const void* ptr, int64_t n_mats, int64_t I, int64_t H) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || n_mats <= 0) return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(I),
+                          static_cast<cuuint64_t>(n_mats)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(H) * 2, static_cast<cuuint64_t>(I * H) * 2};
+    cuuint32_t box[3] = {64u, 128u, 2u};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// The token-row operand with the five box heights 16 << j.
+bool make_tmap_rows(CUtensorMap* maps, const void* ptr, int64_t rows, int64_t cols) {
+    for (int j = 0; j < kNumBoxSizes; ++j)
+        if (!make_tmap(&maps[j], ptr, rows, cols, 16 << j)) return false;
+    return true;
+}
+
 // ------------------------------------------------------------------ problem checks
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -140,14 +164,49 @@ float effective_clip(const moe_problem* p) {
 }
 
 
-// Token-row tile width for the expert GEMMs, from the mean rows per expert.
+int env_int(const char* name, int dflt) {
+    const char* e = std::getenv(name);
+    return e ? std::atoi(e) : dflt;
+}
+
+bool nmax_supported(int n) {
+    return n == 16 || n == 32 || n == 64 || n == 128 || n == 160 || n == 256;
+}
+
+// Token-row tile width (MMA N) of the expert GEMMs, from the mean rows per
+// expert: small batches get narrow tiles (deep weight pipelines, little
+// padding); prefill-sized experts (~100-200 rows) get 160, which leaves room
+// for a 4-deep pipeline of gate+up weight tiles; larger segments get 256.
+// MOE_NMAX in the environment overrides it (tuning knob).
 int pick_nmax(double mean_rows) {
-    if (mean_rows >= 96.0) return 256;
+    static const int forced = [] {
+        const int v = env_int("MOE_NMAX", 0);
+        return nmax_supported(v) ? v : 0;
+    }();
+    if (forced) return forced;
+    if (mean_rows >= 200.0) return 256;
+    if (mean_rows >= 96.0) return 160;
     if (mean_rows >= 48.0) return 128;
-    if (mean_rows >= 12.0) return 64;
+    if (mean_rows >= 24.0) return 64;
+    if (mean_rows >= 12.0) return 32;
     return 16;
 }
+
+// 128-row weight sub-tiles per down-projection tile: two (one 256-row weight
+// box per stage, half the token-tile re-reads) while the two accumulators still
+// fit twice in TMEM (NMAX <= 128), else one so the epilogue stays overlapped
+// with the next tile's main loop.  MOE_DOWN_MB overrides.
+int pick_down_mb(int nmax) {
+    static const int forced = [] {
+        const int v = env_int("MOE_DOWN_MB", 0);
+        return (v == 1 || v == 2) ? v : 0;
+    }();
+    if (forced) return forced;
+    return nmax <= 128 ? 2 : 1;
+}
+
 constexpr int kLogitsNmax = 64;
+constexpr int kLogitsMb = 2;
 
 // ------------------------------------------------------------------ workspace layout
 
@@ -231,41 +290,68 @@ T* at(void* ws, size_t off) {
 
 // ------------------------------------------------------------------ GEMM launch
 
-template <int EPI, int NMAX>
+template <int EPI, int NMAX, int MB>
 int32_t launch_gemm_n(const GemmArgs& a, int grid, cudaStream_t s, const char* name) {
-    using C = GemmCfg<EPI, NMAX>;
+    using C = GemmCfg<EPI, NMAX, MB>;
     int dev = 0;
     cudaGetDevice(&dev);
     static std::atomic<uint64_t> configured{0};
     const uint64_t bit = (dev < 64) ? (1ull << dev) : 0;
     if (!bit || !(configured.load() & bit)) {
-        if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI, NMAX>,
+        if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI, NMAX, MB>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::kSmemBytes) != cudaSuccess)
             return MOE_ERR_CUDA;
         configured.fetch_or(bit);
     }
-    MOE_LAUNCH(name, s, grouped_gemm_kernel<EPI, NMAX><<<grid, C::kThreads, C::kSmemBytes, s>>>(a));
+    MOE_LAUNCH(name, s,
+               grouped_gemm_kernel<EPI, NMAX, MB><<<grid, C::kThreads, C::kSmemBytes, s>>>(a));
     return MOE_OK;
 }
 
-template <int EPI>
-int32_t launch_gemm(int nmax, const GemmArgs& a, int64_t max_tiles, cudaStream_t s,
-                    const char* name) {
-    int grid = static_cast<int>(std::min<int64_t>(sm_count(), std::max<int64_t>(1, max_tiles)));
+template <int EPI, int MB>
+int32_t launch_gemm_mb(int nmax, const GemmArgs& a, int grid, cudaStream_t s, const char* name) {
     switch (nmax) {
-        case 16: return launch_gemm_n<EPI, 16>(a, grid, s, name);
-        case 64: return launch_gemm_n<EPI, 64>(a, grid, s, name);
-        case 128: return launch_gemm_n<EPI, 128>(a, grid, s, name);
-        case 256: return launch_gemm_n<EPI, 256>(a, grid, s, name);
+        case 16: return launch_gemm_n<EPI, 16, MB>(a, grid, s, name);
+        case 32: return launch_gemm_n<EPI, 32, MB>(a, grid, s, name);
+        case 64: return launch_gemm_n<EPI, 64, MB>(a, grid, s, name);
+        case 128: return launch_gemm_n<EPI, 128, MB>(a, grid, s, name);
+        case 160: return launch_gemm_n<EPI, 160, MB>(a, grid, s, name);
+        case 256: return launch_gemm_n<EPI, 256, MB>(a, grid, s, name);
         default: return MOE_ERR_UNSUPPORTED;
     }
 }
 
+// Launch with a persistent grid of min(#SMs, tiles) CTAs.
+template <int EPI>
+int32_t launch_gemm(int nmax, int mb, const GemmArgs& a, int64_t max_tiles, cudaStream_t s,
+                    const char* name) {
+    int grid = static_cast<int>(std::min<int64_t>(sm_count(), std::max<int64_t>(1, max_tiles)));
+    if constexpr (EPI == EPI_SWIGLU) {
+        return launch_gemm_mb<EPI, 2>(nmax, a, grid, s, name);
+    } else if constexpr (EPI == EPI_DOWN_STORE) {
+        return launch_gemm_mb<EPI, 1>(nmax, a, grid, s, name);
+    } else if constexpr (EPI == EPI_LOGITS) {
+        if (nmax != kLogitsNmax) return MOE_ERR_UNSUPPORTED;
+        if (mb == 2) return launch_gemm_n<EPI, kLogitsNmax, 2>(a, grid, s, name);
+        return launch_gemm_n<EPI, kLogitsNmax, 1>(a, grid, s, name);
+    } else {
+        if (mb == 2) return launch_gemm_mb<EPI, 2>(nmax, a, grid, s, name);
+        return launch_gemm_mb<EPI, 1>(nmax, a, grid, s, name);
+    }
+}
+
 // Upper bound on tiles of a schedule: sum over segments of ceil(rows/nmax)
-// <= rows_total/nmax + nseg, times weight blocks.
-int64_t max_tiles(int64_t rows_total, int nseg, int nmax, int64_t m_total) {
-    return (rows_total / nmax + nseg) * ((m_total + 127) / 128);
+// <= rows_total/nmax + nseg, times weight blocks of rows_per_tile rows.
+int64_t max_tiles(int64_t rows_total, int nseg, int nmax, int64_t m_total,
+                  int64_t rows_per_tile = 128) {
+    return (rows_total / nmax + nseg) * ((m_total + rows_per_tile - 1) / rows_per_tile);
+}
+
+// L2 cache hints on the GEMM operand loads (MOE_L2_HINTS=0 turns them off).
+int l2_hints() {
+    static const int v = env_int("MOE_L2_HINTS", 1) ? 1 : 0;
+    return v;
 }
 
 GemmArgs base_args(int32_t* status) {
@@ -273,6 +359,7 @@ GemmArgs base_args(int32_t* status) {
     std::memset(&a, 0, sizeof(a));
     a.special_seg = -1;
     a.clip = INFINITY;
+    a.l2_hints = l2_hints();
     a.status = status;
     return a;
 }
@@ -281,10 +368,11 @@ GemmArgs base_args(int32_t* status) {
 int32_t run_logits_bf16(const moe_problem* p, const void* x, const void* gate_w, float* logits,
                         int32_t* status, cudaStream_t s) {
     GemmArgs a = base_args(status);
-    if (!make_tmap(&a.tmA0, gate_w, p->E, p->H, 128)) return MOE_ERR_CUDA;
-    if (!make_tmap(&a.tmB0, x, p->T, p->H, 16)) return MOE_ERR_CUDA;
+    const int mb = (p->E > 128) ? kLogitsMb : 1;
+    if (!make_tmap(&a.tmA0, gate_w, p->E, p->H, 128 * mb)) return MOE_ERR_CUDA;
+    if (!make_tmap_rows(a.tmB0, x, p->T, p->H)) return MOE_ERR_CUDA;
     a.tmA1 = a.tmA0;
-    a.tmB1 = a.tmB0;
+    for (int j = 0; j < kNumBoxSizes; ++j) a.tmB1[j] = a.tmB0[j];
     a.sched = nullptr;
     a.single_rows = static_cast<int32_t>(p->T);
     a.single_chunk_len = kLogitsNmax;
@@ -293,7 +381,8 @@ int32_t run_logits_bf16(const moe_problem* p, const void* x, const void* gate_w,
     a.M_total = p->E;
     a.out = logits;
     a.out_ld = p->E;
-    return launch_gemm<EPI_LOGITS>(kLogitsNmax, a, max_tiles(p->T, 1, kLogitsNmax, p->E), s,
+    return launch_gemm<EPI_LOGITS>(kLogitsNmax, mb, a,
+                                   max_tiles(p->T, 1, kLogitsNmax, p->E, 128 * mb), s,
                                    "router_logits_gemm");
 }
 
@@ -404,7 +493,7 @@ int32_t run_dispatch(const moe_problem* p, const int32_t* idx, const float* topk
                dispatch_count_kernel<<<nch, kPermTokens, 0, s>>>(idx, p->T, p->E, p->top_k, hist,
                                                                  status));
     MOE_LAUNCH("dispatch_scan", s,
-               dispatch_scan_kernel<<<1, 256, 0, s>>>(hist, static_cast<int>(nch), p->E, p->T,
+               dispatch_scan_kernel<<<1, 512, 0, s>>>(hist, static_cast<int>(nch), p->E, p->T,
                                                       p->top_k, p->num_shared, base, counts,
                                                       offsets, sched_gu, nmax_gu, sched_dn,
                                                       nmax_dn));
@@ -555,31 +644,30 @@ int32_t moe_grouped_swiglu_ffn(const moe_problem* p, const void* x_perm, int64_t
     __nv_bfloat16* h = at<__nv_bfloat16>(ws, L.h_perm);
     {
         GemmArgs a = base_args(status);
-        if (!make_tmap(&a.tmA0, wb, static_cast<int64_t>(n_groups) * 3 * I, H, 128))
+        if (!make_tmap_gateup(&a.tmA0, wb, static_cast<int64_t>(n_groups) * 3, I, H))
             return MOE_ERR_CUDA;
-        if (!make_tmap(&a.tmB0, xb, rows, H, 16)) return MOE_ERR_CUDA;
+        if (!make_tmap_rows(a.tmB0, xb, rows, H)) return MOE_ERR_CUDA;
         a.tmA1 = a.tmA0;
-        a.tmB1 = a.tmB0;
+        for (int j = 0; j < kNumBoxSizes; ++j) a.tmB1[j] = a.tmB0[j];
         a.sched = sg;
         a.nseg = n_groups;
         a.K = static_cast<int32_t>(H);
         a.M_total = static_cast<int32_t>(I);
-        a.a_seg_stride = static_cast<int32_t>(3 * I);
+        a.a_seg_stride = 3;  // matrices per expert
         a.a_off0 = 0;
-        a.a_off1 = static_cast<int32_t>(I);
         a.out = h;
         a.out_ld = static_cast<int32_t>(I);
         a.clip = effective_clip(p);
-        MOE_TRY(launch_gemm<EPI_SWIGLU>(nmax, a, max_tiles(rows, n_groups, nmax, I), s,
+        MOE_TRY(launch_gemm<EPI_SWIGLU>(nmax, 2, a, max_tiles(rows, n_groups, nmax, I), s,
                                         "expert_gate_up_gemm"));
     }
     {
         GemmArgs a = base_args(status);
         if (!make_tmap(&a.tmA0, wb, static_cast<int64_t>(n_groups) * 3 * I, H, 64))
             return MOE_ERR_CUDA;
-        if (!make_tmap(&a.tmB0, h, rows, I, 16)) return MOE_ERR_CUDA;
+        if (!make_tmap_rows(a.tmB0, h, rows, I)) return MOE_ERR_CUDA;
         a.tmA1 = a.tmA0;
-        a.tmB1 = a.tmB0;
+        for (int j = 0; j < kNumBoxSizes; ++j) a.tmB1[j] = a.tmB0[j];
         a.sched = sd;
         a.nseg = n_groups;
         a.K = static_cast<int32_t>(I);
@@ -589,7 +677,7 @@ int32_t moe_grouped_swiglu_ffn(const moe_problem* p, const void* x_perm, int64_t
         a.out = y_perm;
         a.out_ld = static_cast<int32_t>(H);
         a.out_f32 = p->dtype == MOE_F32 ? 1 : 0;
-        MOE_TRY(launch_gemm<EPI_DOWN_STORE>(nmax, a, max_tiles(rows, n_groups, nmax, H), s,
+        MOE_TRY(launch_gemm<EPI_DOWN_STORE>(nmax, 1, a, max_tiles(rows, n_groups, nmax, H), s,
                                             "expert_down_gemm"));
     }
     return MOE_OK;
@@ -694,40 +782,39 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
     const int nseg = static_cast<int>(E + S);
     {
         GemmArgs a = base_args(status);
-        if (!make_tmap(&a.tmA0, ew, E * 3 * I, H, 128)) return MOE_ERR_CUDA;
-        if (!make_tmap(&a.tmB0, x_perm, T * k, H, 16)) return MOE_ERR_CUDA;
+        if (!make_tmap_gateup(&a.tmA0, ew, E * 3, I, H)) return MOE_ERR_CUDA;
+        if (!make_tmap_rows(a.tmB0, x_perm, T * k, H)) return MOE_ERR_CUDA;
         if (S) {
-            if (!make_tmap(&a.tmA1, sw, 3 * I, H, 128)) return MOE_ERR_CUDA;
-            if (!make_tmap(&a.tmB1, x_b, T, H, 16)) return MOE_ERR_CUDA;
+            if (!make_tmap_gateup(&a.tmA1, sw, 3, I, H)) return MOE_ERR_CUDA;
+            if (!make_tmap_rows(a.tmB1, x_b, T, H)) return MOE_ERR_CUDA;
         } else {
             a.tmA1 = a.tmA0;
-            a.tmB1 = a.tmB0;
+            for (int j = 0; j < kNumBoxSizes; ++j) a.tmB1[j] = a.tmB0[j];
         }
         a.sched = sg;
         a.nseg = nseg;
         a.special_seg = S ? static_cast<int32_t>(E) : -1;
         a.K = static_cast<int32_t>(H);
         a.M_total = static_cast<int32_t>(I);
-        a.a_seg_stride = static_cast<int32_t>(3 * I);
+        a.a_seg_stride = 3;  // matrices per expert
         a.a_off0 = 0;
-        a.a_off1 = static_cast<int32_t>(I);
         a.out = h;
         a.out_ld = static_cast<int32_t>(I);
         a.clip = effective_clip(p);
-        MOE_TRY(launch_gemm<EPI_SWIGLU>(nmax, a, max_tiles(h_rows, nseg, nmax, I), s,
+        MOE_TRY(launch_gemm<EPI_SWIGLU>(nmax, 2, a, max_tiles(h_rows, nseg, nmax, I), s,
                                         "expert_gate_up_gemm"));
     }
     // 5. grouped down GEMM, routing weight + scatter-add into the fp32 accumulator
     {
         GemmArgs a = base_args(status);
         if (!make_tmap(&a.tmA0, ew, E * 3 * I, H, 64)) return MOE_ERR_CUDA;
-        if (!make_tmap(&a.tmB0, h, h_rows, I, 16)) return MOE_ERR_CUDA;
+        if (!make_tmap_rows(a.tmB0, h, h_rows, I)) return MOE_ERR_CUDA;
         if (S) {
             if (!make_tmap(&a.tmA1, sw, 3 * I, H, 64)) return MOE_ERR_CUDA;
         } else {
             a.tmA1 = a.tmA0;
         }
-        a.tmB1 = a.tmB0;
+        for (int j = 0; j < kNumBoxSizes; ++j) a.tmB1[j] = a.tmB0[j];
         a.sched = sd;
         a.nseg = nseg;
         a.special_seg = S ? static_cast<int32_t>(E) : -1;
@@ -741,7 +828,9 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
         a.row_token = src;
         a.row_weight = row_w;
         a.routed_rows = static_cast<int32_t>(T * k);
-        MOE_TRY(launch_gemm<EPI_DOWN_ATOMIC>(nmax, a, max_tiles(h_rows, nseg, nmax, H), s,
+        const int mb = pick_down_mb(nmax);
+        MOE_TRY(launch_gemm<EPI_DOWN_ATOMIC>(nmax, mb, a,
+                                             max_tiles(h_rows, nseg, nmax, H, 128 * mb), s,
                                              "expert_down_combine_gemm"));
     }
     // 6. output cast

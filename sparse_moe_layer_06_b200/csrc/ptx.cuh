@@ -1,7 +1,7 @@
 // ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarriers, TMA tile loads,
 // tcgen05 (TMEM allocation, MMA issue, commit, TMEM loads) and fences.
 //
-// Every wait here is bounded: it gives up after kMaxWaitNs of wall time (or as
+// Every wait here is bounded: it gives up after kMaxWaitCycles SM cycles (or as
 // soon as the CTA-wide abort flag is raised), so a lost arrival can never hang
 // the GPU.  Callers turn a failed wait into an error word the host can read.
 #pragma once
@@ -12,18 +12,13 @@
 namespace moe {
 namespace ptx {
 
-// Upper bound on any single barrier wait (1 s); no legitimate wait in these
+// Upper bound on any single barrier wait, in SM clock cycles (about 2 s at the
+// 1965 MHz maximum clock, longer at lower clocks); no legitimate wait in these
 // kernels comes within several orders of magnitude of it.
-constexpr uint64_t kMaxWaitNs = 1000000000ull;
+constexpr uint64_t kMaxWaitCycles = 4000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
 }
 
 __device__ __forceinline__ bool elect_one_lane() {
@@ -66,19 +61,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
 }
 
 // Bounded wait for the phase with the given parity to complete.  Returns false
-// if the wait timed out or the CTA abort flag was raised meanwhile.
+// if the wait timed out or the CTA abort flag was raised meanwhile.  The fast
+// path is a bare try_wait; the cycle counter is only read between batches of
+// polls so that it never sits on the critical path of a completing phase.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           const volatile int* abort_flag) {
     const uint32_t addr = smem_u32(bar);
     if (mbar_try_wait(addr, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    uint32_t iter = 0;
+    const uint64_t t0 = clock64();
     while (true) {
-        if (mbar_try_wait(addr, parity)) return true;
-        if ((++iter & 31u) == 0) {
-            if (abort_flag && *abort_flag) return false;
-            if (globaltimer_ns() - t0 > kMaxWaitNs) return false;
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i) {
+            if (mbar_try_wait(addr, parity)) return true;
         }
+        if (abort_flag && *abort_flag) return false;
+        if (static_cast<uint64_t>(clock64()) - t0 > kMaxWaitCycles) return false;
     }
 }
 
@@ -99,9 +96,27 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
         : "memory");
 }
 
+// 3D tiled bulk tensor load global -> shared (coordinates innermost first).
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m, int32_t c0,
+                                            int32_t c1, int32_t c2, uint64_t* bar,
+                                            uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_"
+        "hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar)),
+        "l"(policy)
+        : "memory");
+}
+
 __device__ __forceinline__ uint64_t policy_evict_first() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ uint64_t policy_evict_normal() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
     return p;
 }
 

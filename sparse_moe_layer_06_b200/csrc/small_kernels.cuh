@@ -150,79 +150,100 @@ __global__ void dispatch_count_kernel(const int32_t* __restrict__ idx, int64_t T
     }
 }
 
-// Fill a tile schedule (see SchedPtrs) for nseg segments from per-segment
-// row counts; run by one thread.  Segment s covers rows [row0(s), row0(s)+rows(s)).
-__device__ void fill_schedule(int32_t* sched, int nseg, int nmax, const int32_t* seg_rows,
-                              const int32_t* seg_b_row0, const int32_t* seg_out_row0) {
-    const SchedPtrs sp = sched_ptrs(sched, nseg);
-    int32_t* prefix = const_cast<int32_t*>(sp.prefix);
-    int32_t* b_row0 = const_cast<int32_t*>(sp.b_row0);
-    int32_t* out_row0 = const_cast<int32_t*>(sp.out_row0);
-    int32_t* rows = const_cast<int32_t*>(sp.rows);
-    int32_t* chunk_len = const_cast<int32_t*>(sp.chunk_len);
-    int acc = 0;
-    for (int s = 0; s < nseg; ++s) {
-        const int r = seg_rows[s];
-        const int chunks = (r + nmax - 1) / nmax;
-        int cl = 16;
-        if (chunks > 0) {
-            cl = (r + chunks - 1) / chunks;
-            cl = (cl + 15) & ~15;
-        }
-        prefix[s] = acc;
-        b_row0[s] = seg_b_row0[s];
-        out_row0[s] = seg_out_row0[s];
-        rows[s] = r;
-        chunk_len[s] = cl;
-        acc += chunks;
+// Exclusive prefix sum over the CTA (blockDim.x a multiple of 32, <= 1024).
+// `s_warp` is 32 ints of shared scratch; every thread must call it.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nwarps = blockDim.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
     }
-    prefix[nseg] = acc;
-}
-
-// Pass 2 (one CTA): per-chunk bases, expert counts and offsets, and the tile
-// schedules of the gate/up and down GEMMs (routed experts, then the shared
-// expert as one more segment when present).
-__global__ void dispatch_scan_kernel(const int32_t* __restrict__ hist, int nchunks, int E,
-                                     int64_t T, int k, int num_shared,
-                                     int32_t* __restrict__ base, int32_t* __restrict__ counts,
-                                     int32_t* __restrict__ offsets, int32_t* sched_gu, int nmax_gu,
-                                     int32_t* sched_dn, int nmax_dn) {
-    __shared__ int32_t s_cnt[kMaxExperts + 1];
-    __shared__ int32_t s_rows[kMaxExperts + 1], s_b0[kMaxExperts + 1], s_o0[kMaxExperts + 1],
-        s_o0b[kMaxExperts + 1];
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int running = 0;
-        for (int c = 0; c < nchunks; ++c) {
-            const int v = hist[static_cast<size_t>(c) * E + e];
-            base[static_cast<size_t>(c) * E + e] = running;
-            running += v;
+    if (lane == 31) s_warp[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < nwarps ? s_warp[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
         }
-        s_cnt[e] = running;
-        counts[e] = running;
+        s_warp[lane] = w;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        int acc = 0;
-        for (int e = 0; e < E; ++e) {
-            offsets[e] = acc;
-            s_rows[e] = s_cnt[e];
-            s_b0[e] = acc;
-            s_o0[e] = acc;
-            s_o0b[e] = acc;
-            acc += s_cnt[e];
+    const int result = (warp > 0 ? s_warp[warp - 1] : 0) + x - v;
+    if (total) *total = s_warp[nwarps - 1];
+    __syncthreads();
+    return result;
+}
+
+// Tile schedule entry of one segment (see SchedPtrs): chunk count and chunk
+// length for rows split into chunks of at most nmax rows (multiples of 16).
+__device__ __forceinline__ void segment_chunks(int rows, int nmax, int* chunks, int* chunk_len) {
+    const int c = (rows + nmax - 1) / nmax;
+    int cl = 16;
+    if (c > 0) cl = (((rows + c - 1) / c) + 15) & ~15;
+    *chunks = c;
+    *chunk_len = cl;
+}
+
+// Pass 2 (one CTA of 512 threads; thread s handles expert / segment s): per-chunk
+// bases, expert counts and offsets, and the tile schedules of the gate/up and
+// down GEMMs (routed experts, then the shared expert as one more segment).
+__global__ void __launch_bounds__(512) dispatch_scan_kernel(
+    const int32_t* __restrict__ hist, int nchunks, int E, int64_t T, int k, int num_shared,
+    int32_t* __restrict__ base, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+    int32_t* sched_gu, int nmax_gu, int32_t* sched_dn, int nmax_dn) {
+    __shared__ int s_warp[32];
+    const int tid = threadIdx.x;
+    int cnt = 0;
+    if (tid < E) {
+        int running = 0;
+#pragma unroll 4
+        for (int c = 0; c < nchunks; ++c) {
+            const int v = hist[static_cast<size_t>(c) * E + tid];
+            base[static_cast<size_t>(c) * E + tid] = running;
+            running += v;
         }
-        offsets[E] = acc;
-        const int routed = static_cast<int>(T * k);
-        int nseg = E;
-        if (num_shared) {
-            s_rows[E] = static_cast<int>(T);
-            s_b0[E] = 0;         // gate/up: the shared expert reads x itself
-            s_o0[E] = routed;    // its h rows follow the routed rows
-            s_o0b[E] = routed;   // down: B rows are those same h rows
-            nseg = E + 1;
+        cnt = running;
+        counts[tid] = cnt;
+    }
+    int total = 0;
+    const int off = block_exclusive_scan(cnt, s_warp, &total);
+    if (tid < E) offsets[tid] = off;
+    if (tid == 0) offsets[E] = total;
+
+    const int routed = static_cast<int>(T * k);
+    const int nseg = E + (num_shared ? 1 : 0);
+    int rows = 0, b0_gu = 0, b0_dn = 0, o0 = 0;
+    if (tid < E) {
+        rows = cnt;
+        b0_gu = b0_dn = o0 = off;
+    } else if (tid == E && num_shared) {
+        rows = static_cast<int>(T);
+        b0_gu = 0;       // gate/up: the shared expert reads x itself
+        b0_dn = routed;  // down: its h rows follow the routed rows
+        o0 = routed;
+    }
+    const bool active = tid < nseg;
+    for (int which = 0; which < 2; ++which) {
+        int32_t* sched = which == 0 ? sched_gu : sched_dn;
+        const int nmax = which == 0 ? nmax_gu : nmax_dn;
+        int chunks = 0, cl = 16;
+        if (active) segment_chunks(rows, nmax, &chunks, &cl);
+        int tot = 0;
+        const int pre = block_exclusive_scan(chunks, s_warp, &tot);
+        if (sched && active) {
+            const SchedPtrs sp = sched_ptrs(sched, nseg);
+            const_cast<int32_t*>(sp.prefix)[tid] = pre;
+            const_cast<int32_t*>(sp.b_row0)[tid] = which == 0 ? b0_gu : b0_dn;
+            const_cast<int32_t*>(sp.out_row0)[tid] = o0;
+            const_cast<int32_t*>(sp.rows)[tid] = rows;
+            const_cast<int32_t*>(sp.chunk_len)[tid] = cl;
+            if (tid == 0) const_cast<int32_t*>(sp.prefix)[nseg] = tot;
         }
-        if (sched_gu) fill_schedule(sched_gu, nseg, nmax_gu, s_rows, s_b0, s_o0);
-        if (sched_dn) fill_schedule(sched_dn, nseg, nmax_dn, s_rows, s_o0b, s_o0b);
     }
 }
 
