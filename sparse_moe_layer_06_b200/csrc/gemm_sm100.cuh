@@ -15,11 +15,14 @@
 // batch (a couple of rows per expert: N = 16) and a prefill batch (hundreds of
 // rows per expert: N up to 256) without padding every expert to 128 rows.
 //
-// Roles (192 threads = 6 warps, one CTA per SM, persistent over tiles):
+// Roles (320 threads = 10 warps, one CTA per SM, persistent over tiles):
 //   warp 0      TMA producer: fills a STAGES-deep shared-memory ring
 //   warp 1      TMEM owner + MMA issuer (one thread issues tcgen05.mma)
-//   warps 2..5  epilogue: tcgen05.ld the fp32 accumulator, apply the epilogue,
-//               store to global memory; each warp owns one 32-lane TMEM quarter
+//   warps 2..9  epilogue: tcgen05.ld the fp32 accumulator, apply the epilogue,
+//               store to global memory.  A warp may only read the 32-lane TMEM
+//               quarter (warp % 4); two warps share each quarter and take
+//               alternate 16-column chunks, so every scheduler has two
+//               independent epilogue instruction streams to interleave.
 // The accumulator is double-buffered in TMEM when it fits, so the epilogue of
 // tile i overlaps the main loop of tile i+1.
 //
@@ -84,8 +87,9 @@ constexpr int kNumBoxSizes = 5;
 
 struct GemmArgs {
     // A (weights).  EPI_SWIGLU: 3D map {H, I, matrices} with a {64, 128, 2} box
-    // (gate and up tiles of one expert in one copy); EPI_DOWN_*: 2D map over
-    // the [rows, H] view with a {64, 64} box; EPI_LOGITS: 2D {64, 128*MB}.
+    // (gate and up tiles of one expert in one copy); EPI_DOWN_*: 3D map
+    // {64, rows, H/64} of the [rows, H] view (strides H*2 and 128 bytes) with a
+    // {64, 64, 2*MB} box; EPI_LOGITS: 2D {64, 128*MB}.
     CUtensorMap tmA0;                // ordinary segments
     CUtensorMap tmA1;                // the special segment (shared expert)
     CUtensorMap tmB0[kNumBoxSizes];  // B (token rows), box {64, 16 << j}
@@ -143,15 +147,17 @@ struct GemmCfg {
     // tail: 1 KB alignment slack + barriers/flags + the schedule (5 arrays)
     // + (EPI_DOWN_ATOMIC) two buffers of the token and weight of each column
     static constexpr int kBarrierBytes = 512;
-    static constexpr int kSchedBytes = 5 * (kMaxSegments + 1) * 4;
+    // (rounded to 128 bytes so that what follows stays 128-byte aligned)
+    static constexpr int kSchedBytes = (5 * (kMaxSegments + 1) * 4 + 127) / 128 * 128;
     static constexpr int kMetaBytes = (EPI == EPI_DOWN_ATOMIC) ? 2 * NMAX * 8 : 0;
+    static constexpr int kEpiWarps = 8;
     static constexpr int kTailBytes = 1024 + kBarrierBytes + kSchedBytes + kMetaBytes;
     static constexpr int kMaxSmem = 227 * 1024;
     static constexpr int kStagesRaw = (kMaxSmem - kTailBytes) / kStageBytes;
     static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
     static_assert(kStages >= 2, "pipeline depth");
     static constexpr int kSmemBytes = kStages * kStageBytes + kTailBytes;
-    static constexpr int kThreads = 192;
+    static constexpr int kThreads = 32 * (2 + kEpiWarps);
 };
 
 struct TileInfo {
@@ -194,12 +200,20 @@ __device__ __forceinline__ bool decode_tile(int t, int nblk, int nseg, const Sme
     return n > 0;
 }
 
+// Reciprocal of d >= 1 with the hardware approximation (relative error ~2^-23;
+// 1/inf = 0, the correct limit of the SiLU gate).
+__device__ __forceinline__ float fast_rcp(float d) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(d));
+    return r;
+}
+
 __device__ __forceinline__ float clamp_keep_nan(float v, float lim) {
     return v > lim ? lim : (v < -lim ? -lim : v);
 }
 
 template <int EPI, int NMAX, int MB>
-__global__ void __launch_bounds__(192, 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs args) {
+__global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs args) {
     using C = GemmCfg<EPI, NMAX, MB>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned ring (the 128-byte swizzle atoms need it)
@@ -245,11 +259,11 @@ __global__ void __launch_bounds__(192, 1) grouped_gemm_kernel(const __grid_const
         }
         for (int a = 0; a < 2; ++a) {
             ptx::mbar_init(&accf_bar[a], 1);
-            ptx::mbar_init(&acce_bar[a], 4);
+            ptx::mbar_init(&acce_bar[a], C::kEpiWarps);
         }
         ptx::mbar_init(final_bar, 1);
-        ptx::mbar_init(&metaf_bar[0], 4);
-        ptx::mbar_init(&metaf_bar[1], 4);
+        ptx::mbar_init(&metaf_bar[0], C::kEpiWarps);
+        ptx::mbar_init(&metaf_bar[1], C::kEpiWarps);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -311,17 +325,10 @@ __global__ void __launch_bounds__(192, 1) grouped_gemm_kernel(const __grid_const
                     armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
                     const int k0 = kb * 64;
                     if constexpr (C::kDown) {
-                        // MN-major A: per sub-tile two 64(H) x 64(K) boxes side
-                        // by side in H
-                        const int krow = a_base + args.a_off0 + k0;
-#pragma unroll
-                        for (int j = 0; j < MB; ++j) {
-                            const int h0 = (ti.blk * MB + j) * 128;
-                            ptx::tma_load_2d(sA + j * C::kATileBytes, tA, h0, krow,
-                                             &full_bar[stage], pol_w);
-                            ptx::tma_load_2d(sA + j * C::kATileBytes + 8192, tA, h0 + 64, krow,
-                                             &full_bar[stage], pol_w);
-                        }
+                        // MN-major A: one 3D copy of 2*MB chunks of 64 H-values
+                        // x 64 K-rows, chunk-major in shared memory (8 KB each)
+                        ptx::tma_load_3d(sA, tA, 0, a_base + args.a_off0 + k0,
+                                         ti.blk * 2 * MB, &full_bar[stage], pol_w);
                     } else if constexpr (C::kSwiGLU) {
                         // gate and up tiles (adjacent matrices) in one 3D copy
                         ptx::tma_load_3d(sA, tA, k0, ti.blk * 128, a_base + args.a_off0,
@@ -420,6 +427,7 @@ __global__ void __launch_bounds__(192, 1) grouped_gemm_kernel(const __grid_const
     } else {
         // ------------------------------------------------------------ epilogue
         const int quarter = warp & 3;
+        const int half = (warp - 2) >> 2;  // which of the two warps on this quarter
         const int row_in_tile = quarter * 32 + lane;
         uint32_t acc = 0, acc_phase = 0;
         uint32_t mi = 0, meta_phase = 0;
@@ -429,13 +437,13 @@ __global__ void __launch_bounds__(192, 1) grouped_gemm_kernel(const __grid_const
             int32_t* w_tok = reinterpret_cast<int32_t*>(s_meta) + mi * 2 * NMAX;
             float* w_wt = reinterpret_cast<float*>(w_tok + NMAX);
             if constexpr (EPI == EPI_DOWN_ATOMIC) {
-                // token and routing weight of every column, fetched by the four
-                // epilogue warps together (a quarter each) before the
-                // accumulator is ready, so the loads overlap the main loop.
-                // Two buffers alternate by tile; a warp only refills a buffer
-                // after all four have published the next tile's quarter, i.e.
-                // after all of them finished reading it.
-                for (int c = (warp - 2) * 32 + lane; c < ti.n_valid; c += 128) {
+                // token and routing weight of every column, fetched by the
+                // epilogue warps together before the accumulator is ready, so
+                // the loads overlap the main loop.  Two buffers alternate by
+                // tile; a warp only refills a buffer after all epilogue warps
+                // have published their part of the next tile, i.e. after all
+                // of them finished reading it.
+                for (int c = (warp - 2) * 32 + lane; c < ti.n_valid; c += 32 * C::kEpiWarps) {
                     const int r = ti.out_row + c;
                     int tok;
                     float wt;
@@ -466,36 +474,82 @@ __global__ void __launch_bounds__(192, 1) grouped_gemm_kernel(const __grid_const
             const uint32_t tbase = tmem_base + acc * C::kAccCols +
                                    (static_cast<uint32_t>(quarter * 32) << 16);
             if constexpr (C::kSwiGLU) {
+                // h = silu(clamp(g)) * clamp(u) on this warp's 16-column chunks;
+                // the next chunk's TMEM loads are in flight while one is
+                // computed.  Lanes pair up (i, i+1) so each store is a bf16x2.
                 const int m = ti.blk * 128 + row_in_tile;
-                const bool m_ok = m < args.M_total;
+                const bool m_ok = m < args.M_total;  // I is even: lane pairs agree
+                const bool odd = lane & 1;
+                const int m_pair = m - (odd ? 1 : 0);
                 __nv_bfloat16* hout = reinterpret_cast<__nv_bfloat16*>(args.out);
-                for (int c0 = 0; c0 < ti.n_mma; c0 += 16) {
-                    float g[16], u[16];
-                    ptx::tmem_ld16(tbase + c0, g);
-                    ptx::tmem_ld16(tbase + NMAX + c0, u);
-                    ptx::tmem_ld_wait();
-                    if (m_ok) {
+                auto emit = [&](float (&g)[16], float (&u)[16], int c0) {
+                    float hv[16];
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            if (c0 + j < ti.n_valid) {
-                                const float gg = clamp_keep_nan(g[j], args.clip);
-                                const float uu = clamp_keep_nan(u[j], args.clip);
-                                const float hval = gg / (1.0f + __expf(-gg)) * uu;
-                                hout[static_cast<size_t>(ti.out_row + c0 + j) * args.out_ld + m] =
-                                    __float2bfloat16_rn(hval);
-                            }
+                    for (int j = 0; j < 16; ++j) {
+                        const float gg = clamp_keep_nan(g[j], args.clip);
+                        const float uu = clamp_keep_nan(u[j], args.clip);
+                        // silu(g) = g / (1 + e^-g): approximate exp2 and
+                        // reciprocal (both ~1e-7 relative, far below bf16)
+                        hv[j] = gg * fast_rcp(1.0f + __expf(-gg)) * uu;
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; j += 2) {
+                        // even lane: (my h, partner's h) of column j;
+                        // odd lane: (partner's h, my h) of column j+1
+                        const float mine = odd ? hv[j + 1] : hv[j];
+                        const float send = odd ? hv[j] : hv[j + 1];
+                        const float other = __shfl_xor_sync(0xffffffffu, send, 1);
+                        const int col = c0 + j + (odd ? 1 : 0);
+                        const __nv_bfloat162 pr = odd ? __floats2bfloat162_rn(other, mine)
+                                                      : __floats2bfloat162_rn(mine, other);
+                        if (m_ok && col < ti.n_valid) {
+                            *reinterpret_cast<__nv_bfloat162*>(
+                                hout + static_cast<size_t>(ti.out_row + col) * args.out_ld +
+                                m_pair) = pr;
                         }
                     }
+                };
+                float g0[16], u0[16], g1[16], u1[16];
+                int c0 = half * 16;  // this warp's chunks: c0, c0 + 32, ...
+                if (c0 < ti.n_mma) {
+                    ptx::tmem_ld16(tbase + c0, g0);
+                    ptx::tmem_ld16(tbase + NMAX + c0, u0);
+                    ptx::tmem_ld_wait();
+                    ptx::reg_fence(g0);
+                    ptx::reg_fence(u0);
+                }
+                for (; c0 < ti.n_mma; c0 += 64) {
+                    const bool more1 = c0 + 32 < ti.n_mma;
+                    if (more1) {
+                        ptx::tmem_ld16(tbase + c0 + 32, g1);
+                        ptx::tmem_ld16(tbase + NMAX + c0 + 32, u1);
+                    }
+                    emit(g0, u0, c0);
+                    if (!more1) break;
+                    ptx::tmem_ld_wait();
+                    ptx::reg_fence(g1);
+                    ptx::reg_fence(u1);
+                    const bool more2 = c0 + 64 < ti.n_mma;
+                    if (more2) {
+                        ptx::tmem_ld16(tbase + c0 + 64, g0);
+                        ptx::tmem_ld16(tbase + NMAX + c0 + 64, u0);
+                    }
+                    emit(g1, u1, c0 + 32);
+                    if (!more2) break;
+                    ptx::tmem_ld_wait();
+                    ptx::reg_fence(g0);
+                    ptx::reg_fence(u0);
                 }
             } else {
 #pragma unroll 1
                 for (int sub = 0; sub < MB; ++sub) {
                     const int m = (ti.blk * MB + sub) * 128 + row_in_tile;
                     const bool m_ok = m < args.M_total;
-                    for (int c0 = 0; c0 < ti.n_mma; c0 += 16) {
+                    for (int c0 = half * 16; c0 < ti.n_mma; c0 += 32) {
                         float v[16];
                         ptx::tmem_ld16(tbase + sub * NMAX + c0, v);
                         ptx::tmem_ld_wait();
+                        ptx::reg_fence(v);
                         if constexpr (EPI == EPI_DOWN_ATOMIC) {
                             float* oacc = reinterpret_cast<float*>(args.out);
 #pragma unroll

@@ -132,6 +132,23 @@ bool make_tmap_gateup(CUtensorMap* m, const void* ptr, int64_t n_mats, int64_t I
     return r == CUDA_SUCCESS;
 }
 
+// Down-projection weights [rows, H] (H contiguous) as a 3D tensor {64, rows,
+// H/64}: dim 0 = 64 consecutive H values, dim 1 = the row (stride H*2 bytes),
+// dim 2 = which 64-wide H chunk (stride 128 bytes).  A {64, 64, 2*mb} box is
+// one K-step of 2*mb chunks, laid out chunk by chunk in shared memory.
+bool make_tmap_down(CUtensorMap* m, const void* ptr, int64_t rows, int64_t H, int mb) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || rows <= 0 || H % 64 != 0) return false;
+    cuuint64_t dims[3] = {64u, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(H / 64)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(H) * 2, 128u};
+    cuuint32_t box[3] = {64u, 64u, static_cast<cuuint32_t>(2 * mb)};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // The token-row operand with the five box heights 16 << j.
 bool make_tmap_rows(CUtensorMap* maps, const void* ptr, int64_t rows, int64_t cols) {
     for (int j = 0; j < kNumBoxSizes; ++j)
@@ -192,17 +209,18 @@ int pick_nmax(double mean_rows) {
     return 16;
 }
 
-// 128-row weight sub-tiles per down-projection tile: two (one 256-row weight
-// box per stage, half the token-tile re-reads) while the two accumulators still
-// fit twice in TMEM (NMAX <= 128), else one so the epilogue stays overlapped
-// with the next tile's main loop.  MOE_DOWN_MB overrides.
+// 128-row weight sub-tiles per down-projection tile: two, i.e. one 3D copy of
+// 32 KB of weights per pipeline stage against each token tile, which halves
+// the token-tile re-reads (the down GEMM is bound by the bulk-copy rows it
+// issues).  MOE_DOWN_MB overrides.
 int pick_down_mb(int nmax) {
     static const int forced = [] {
         const int v = env_int("MOE_DOWN_MB", 0);
         return (v == 1 || v == 2) ? v : 0;
     }();
     if (forced) return forced;
-    return nmax <= 128 ? 2 : 1;
+    (void)nmax;
+    return 2;
 }
 
 constexpr int kLogitsNmax = 64;
@@ -663,7 +681,7 @@ int32_t moe_grouped_swiglu_ffn(const moe_problem* p, const void* x_perm, int64_t
     }
     {
         GemmArgs a = base_args(status);
-        if (!make_tmap(&a.tmA0, wb, static_cast<int64_t>(n_groups) * 3 * I, H, 64))
+        if (!make_tmap_down(&a.tmA0, wb, static_cast<int64_t>(n_groups) * 3 * I, H, 1))
             return MOE_ERR_CUDA;
         if (!make_tmap_rows(a.tmB0, h, rows, I)) return MOE_ERR_CUDA;
         a.tmA1 = a.tmA0;
@@ -807,10 +825,11 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
     // 5. grouped down GEMM, routing weight + scatter-add into the fp32 accumulator
     {
         GemmArgs a = base_args(status);
-        if (!make_tmap(&a.tmA0, ew, E * 3 * I, H, 64)) return MOE_ERR_CUDA;
+        const int mb = pick_down_mb(nmax);
+        if (!make_tmap_down(&a.tmA0, ew, E * 3 * I, H, mb)) return MOE_ERR_CUDA;
         if (!make_tmap_rows(a.tmB0, h, h_rows, I)) return MOE_ERR_CUDA;
         if (S) {
-            if (!make_tmap(&a.tmA1, sw, 3 * I, H, 64)) return MOE_ERR_CUDA;
+            if (!make_tmap_down(&a.tmA1, sw, 3 * I, H, mb)) return MOE_ERR_CUDA;
         } else {
             a.tmA1 = a.tmA0;
         }
@@ -828,7 +847,6 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
         a.row_token = src;
         a.row_weight = row_w;
         a.routed_rows = static_cast<int32_t>(T * k);
-        const int mb = pick_down_mb(nmax);
         MOE_TRY(launch_gemm<EPI_DOWN_ATOMIC>(nmax, mb, a,
                                              max_tiles(h_rows, nseg, nmax, H, 128 * mb), s,
                                              "expert_down_combine_gemm"));
