@@ -264,7 +264,7 @@ def main():
     ap.add_argument("--config", default="hy4_prefill", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T of the workload (smaller cases for profiling)")
     ap.add_argument("--experts", type=int, default=None,
@@ -349,27 +349,51 @@ def main():
     status = moe.moe_read_device_status(ws)
     ms_per_step = ms / args.steps
 
-    # ---------------- end to end: host buffers, copies inside the timed region
+    # ---------------- end to end: host buffers, copies inside the timed region.
+    # Each step copies its tokens in from pinned host memory, runs the layer
+    # and copies the output back.  As a serving loop would, steps are
+    # pipelined over two device buffers and three streams (copy-in, compute,
+    # copy-out) so the PCIe copies of one step overlap the layer of another.
     x_host = inp["x"].cpu().pin_memory()
-    out_host = torch.empty(cfg.T, cfg.H, dtype=cfg.dtype).pin_memory()
-    x_dev = torch.empty_like(inp["x"])
-    for _ in range(3):
-        x_dev.copy_(x_host, non_blocking=True)
-        moe.moe_forward(p, x_dev, inp["gate_w"], inp["logit_bias"], inp["expert_w"],
-                        inp["shared_w"], out, idx, w, ws, stream)
-        out_host.copy_(out, non_blocking=True)
+    out_host = [torch.empty(cfg.T, cfg.H, dtype=cfg.dtype).pin_memory() for _ in range(2)]
+    x_dev = [torch.empty_like(inp["x"]) for _ in range(2)]
+    out_dev = [torch.empty_like(out) for _ in range(2)]
+    s_in = torch.cuda.Stream(dev)
+    s_out = torch.cuda.Stream(dev)
+    s_cmp = stream
+    in_done = [torch.cuda.Event() for _ in range(2)]
+    cmp_done = [torch.cuda.Event() for _ in range(2)]
+    out_done = [torch.cuda.Event() for _ in range(2)]
+
+    def e2e_steps(n):
+        for i in range(n):
+            b = i & 1
+            if i >= 2:
+                s_in.wait_event(cmp_done[b])  # the layer is done reading x_dev[b]
+            with torch.cuda.stream(s_in):
+                x_dev[b].copy_(x_host, non_blocking=True)
+            in_done[b].record(s_in)
+            s_cmp.wait_event(in_done[b])
+            if i >= 2:
+                s_cmp.wait_event(out_done[b])  # out_dev[b] was copied out
+            moe.moe_forward(p, x_dev[b], inp["gate_w"], inp["logit_bias"], inp["expert_w"],
+                            inp["shared_w"], out_dev[b], idx, w, ws, s_cmp)
+            cmp_done[b].record(s_cmp)
+            s_out.wait_event(cmp_done[b])
+            with torch.cuda.stream(s_out):
+                out_host[b].copy_(out_dev[b], non_blocking=True)
+            out_done[b].record(s_out)
+
+    e2e_steps(3)
     torch.cuda.synchronize(dev)
     if dist:
         dist.barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
-        x_dev.copy_(x_host, non_blocking=True)
-        moe.moe_forward(p, x_dev, inp["gate_w"], inp["logit_bias"], inp["expert_w"],
-                        inp["shared_w"], out, idx, w, ws, stream)
-        out_host.copy_(out, non_blocking=True)
-    e1.record(stream)
+    e0.record(s_in)
+    e2e_steps(args.e2e_steps)
+    s_out.wait_event(cmp_done[(args.e2e_steps - 1) & 1])
+    e1.record(s_out)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1)
     if dist:
@@ -427,7 +451,7 @@ def main():
         cpu_base = oracle_baseline(cfg, cpu_inp)
 
     h2d = cfg.T * cfg.H * x_host.element_size()
-    d2h = cfg.T * cfg.H * out_host.element_size()
+    d2h = cfg.T * cfg.H * out_host[0].element_size()
     line = {
         "metric": METRIC,
         "value": tokens_per_s,

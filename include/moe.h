@@ -37,8 +37,8 @@
  *    cores.  MOE_F32 - x, weights, outputs fp32; the router runs in fp32 on
  *    CUDA cores, the expert GEMMs run on bf16 copies made on the device.
  *  - Shapes supported: T >= 0 (T == 0 is a no-op), H and I multiples of 64,
- *    1 <= top_k <= E <= 256, num_shared in {0,1}, T*top_k < 2^31.  Anything
- *    else returns MOE_ERR_UNSUPPORTED.
+ *    1 <= top_k <= min(E, 32), E <= 256, num_shared in {0,1},
+ *    T*top_k < 2^31.  Anything else returns MOE_ERR_UNSUPPORTED.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H

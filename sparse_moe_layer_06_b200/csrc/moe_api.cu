@@ -165,7 +165,8 @@ int32_t check_problem(const moe_problem* p) {
     if (p->T < 0) return MOE_ERR_INVALID_ARG;
     if (p->dtype != MOE_F32 && p->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
     if (p->H < 64 || p->H % 64 != 0 || p->I < 64 || p->I % 64 != 0) return MOE_ERR_UNSUPPORTED;
-    if (p->E < 1 || p->E > kMaxExperts || p->top_k < 1 || p->top_k > p->E)
+    // top_k <= 32: the router and the row gather keep one selection per lane
+    if (p->E < 1 || p->E > kMaxExperts || p->top_k < 1 || p->top_k > p->E || p->top_k > 32)
         return MOE_ERR_UNSUPPORTED;
     if (p->num_shared != 0 && p->num_shared != 1) return MOE_ERR_UNSUPPORTED;
     if (p->T * static_cast<int64_t>(p->top_k + p->num_shared) >= (int64_t(1) << 31))
@@ -456,30 +457,44 @@ __global__ void gather_kernel(const TIn* __restrict__ x, int64_t T, int H, int k
         if (my_pos < 0 || my_pos >= n_rows) my_pos = -1;
     }
     constexpr int kElems = 16 / sizeof(TOut);  // elements per 16-byte output vector
+    constexpr int kBatch = 8;  // 16-byte loads in flight per lane before the stores
     const int nvec = H / kElems;
-    for (int v = lane; v < nvec; v += 32) {
-        uint4 packed;
-        uint4 packed_bf16;
-        if constexpr (sizeof(TIn) == sizeof(TOut)) {
-            packed = reinterpret_cast<const uint4*>(x + t * H)[v];
-        } else {
-            // fp32 -> bf16: 8 inputs per output vector
-            const float4 a = reinterpret_cast<const float4*>(x + t * H)[2 * v];
-            const float4 b = reinterpret_cast<const float4*>(x + t * H)[2 * v + 1];
-            __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y);
-            __nv_bfloat162 p1 = __floats2bfloat162_rn(a.z, a.w);
-            __nv_bfloat162 p2 = __floats2bfloat162_rn(b.x, b.y);
-            __nv_bfloat162 p3 = __floats2bfloat162_rn(b.z, b.w);
-            packed.x = *reinterpret_cast<uint32_t*>(&p0);
-            packed.y = *reinterpret_cast<uint32_t*>(&p1);
-            packed.z = *reinterpret_cast<uint32_t*>(&p2);
-            packed.w = *reinterpret_cast<uint32_t*>(&p3);
-            packed_bf16 = packed;
-            if (x_bf16) reinterpret_cast<uint4*>(x_bf16 + t * H)[v] = packed_bf16;
+    for (int v0 = 0; v0 < nvec; v0 += 32 * kBatch) {
+        uint4 packed[kBatch];
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            const int v = v0 + b * 32 + lane;
+            if (v < nvec) {
+                if constexpr (sizeof(TIn) == sizeof(TOut)) {
+                    packed[b] = reinterpret_cast<const uint4*>(x + t * H)[v];
+                } else {
+                    // fp32 -> bf16: 8 inputs per output vector
+                    const float4 a = reinterpret_cast<const float4*>(x + t * H)[2 * v];
+                    const float4 c = reinterpret_cast<const float4*>(x + t * H)[2 * v + 1];
+                    __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y);
+                    __nv_bfloat162 p1 = __floats2bfloat162_rn(a.z, a.w);
+                    __nv_bfloat162 p2 = __floats2bfloat162_rn(c.x, c.y);
+                    __nv_bfloat162 p3 = __floats2bfloat162_rn(c.z, c.w);
+                    packed[b].x = *reinterpret_cast<uint32_t*>(&p0);
+                    packed[b].y = *reinterpret_cast<uint32_t*>(&p1);
+                    packed[b].z = *reinterpret_cast<uint32_t*>(&p2);
+                    packed[b].w = *reinterpret_cast<uint32_t*>(&p3);
+                }
+            }
         }
-        for (int j = 0; j < k; ++j) {
-            const int r = __shfl_sync(0xffffffffu, my_pos, j);
-            if (r >= 0) reinterpret_cast<uint4*>(x_perm + static_cast<int64_t>(r) * H)[v] = packed;
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            const int v = v0 + b * 32 + lane;
+            const bool ok = v < nvec;
+            if constexpr (sizeof(TIn) != sizeof(TOut)) {
+                if (ok && x_bf16) reinterpret_cast<uint4*>(x_bf16 + t * H)[v] = packed[b];
+            }
+            // every lane takes part in the shuffles; only the stores are predicated
+            for (int j = 0; j < k; ++j) {
+                const int r = __shfl_sync(0xffffffffu, my_pos, j);
+                if (ok && r >= 0)
+                    reinterpret_cast<uint4*>(x_perm + static_cast<int64_t>(r) * H)[v] = packed[b];
+            }
         }
     }
     if (acc_zero) {

@@ -68,7 +68,7 @@ def test_workspace_sizes_monotone_and_validated(lib):
     assert moe.moe_workspace_size(big, moe.MOE_CALL_FORWARD) > sizes[moe.MOE_CALL_FORWARD]
     # unsupported shapes report 0
     for bad in (problem(H=100), problem(I=96), problem(E=300), problem(top_k=17),
-                problem(num_shared=2), problem(T=-1)):
+                problem(E=64, top_k=33), problem(num_shared=2), problem(T=-1)):
         assert moe.moe_workspace_size(bad, moe.MOE_CALL_FORWARD) == 0
     assert moe.moe_workspace_size(p, 42) == 0
 
