@@ -174,6 +174,29 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(mine)}
 
 
+# ------------------------------------------------------------------ ranks
+
+def rank_token_seed(rank: int) -> int:
+    """Seed of a rank's token batch: every rank holds the same weights (seeds
+    1..3 of the workload recipe) and its own tokens."""
+    return 1000 * rank
+
+
+def max_over_ranks(value: float, dist=None, device="cpu") -> float:
+    """The slowest rank's time: an all-reduce MAX over the process group (NCCL
+    on GPUs, gloo on CPU), or the value itself on a single process."""
+    if dist is None:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: int, world: int, seconds: float) -> float:
+    """Units all ranks processed divided by the (max over ranks) time."""
+    return world * units_per_rank / seconds
+
+
 # ------------------------------------------------------------------ CPU oracle baseline
 
 def oracle_baseline(cfg, cpu_inp, budget_s=12.0, max_tokens=256):
@@ -298,7 +321,7 @@ def main():
 
     # identical weights on every rank, a different token batch per rank
     inp = make_inputs(cfg.with_tokens(1), seed=0, device=dev)
-    inp["x"] = make_x(cfg, seed=1000 * rank, device=dev)
+    inp["x"] = make_x(cfg, seed=rank_token_seed(rank), device=dev)
     if cfg.skew_bias:
         from sparse_moe_layer_06_b200.workloads import skew_logit_bias
         inp["logit_bias"] = skew_logit_bias(cfg.E).to(dev)
@@ -341,11 +364,7 @@ def main():
         dist.barrier()
     kernel_times = moe.moe_profile_stop()
     clocks.stop()
-    ms = ev0.elapsed_time(ev1)
-    if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), dist, dev)
     status = moe.moe_read_device_status(ws)
     ms_per_step = ms / args.steps
 
@@ -395,11 +414,8 @@ def main():
     s_out.wait_event(cmp_done[(args.e2e_steps - 1) & 1])
     e1.record(s_out)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
         dist.barrier()
 
     if rank != 0:
@@ -414,7 +430,7 @@ def main():
     idx_cpu = idx.cpu()
     flops, bytes_, touched = layer_counts(cfg, idx_cpu)
     t_s = ms_per_step / 1e3
-    tokens_per_s = world * cfg.T / t_s
+    tokens_per_s = whole_job_rate(cfg.T, world, t_s)
     roof_t = max(flops / (tf_peak * 1e12), bytes_ / (hbm_peak * 1e9))
     layer_frac = roof_t / t_s
     roof_t_nominal = max(flops / 2250e12, bytes_ / 8000e9)
@@ -478,7 +494,8 @@ def main():
         "kernels": per_kernel,
         "cpu_baseline": cpu_base,
         "clocks": clocks.summary(wall1 - ms / 1e3, wall1),
-        "e2e": {"value": world * cfg.T * args.e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+        "e2e": {"value": whole_job_rate(cfg.T * args.e2e_steps, world, e2e_ms / 1e3),
+                "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
         "device_status": status,
