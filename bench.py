@@ -72,14 +72,16 @@ def gate_up_counts(cfg, touched):
     return flops, bytes_
 
 
-def down_counts(cfg, touched):
-    """One launch of the grouped down GEMM + weighted scatter-add: down weights
-    of every touched expert (+ shared), h read once, the fp32 accumulator read
-    and written once per token."""
+def down_counts(cfg, touched, scatter_add=False):
+    """One launch of the grouped down GEMM: down weights of every touched expert
+    (+ shared) and h read once; then either the weighted bf16 rows written once
+    (store epilogue) or the fp32 token accumulator read and written once
+    (scatter-add epilogue)."""
     T, H, I, k, S = cfg.T, cfg.H, cfg.I, cfg.top_k, cfg.num_shared
     rows = T * (k + S)
     flops = 2 * rows * H * I
-    bytes_ = (touched + S) * I * H * 2 + rows * I * 2 + 2 * T * H * 4
+    out_bytes = 2 * T * H * 4 if scatter_add else rows * H * 2
+    bytes_ = (touched + S) * I * H * 2 + rows * I * 2 + out_bytes
     return flops, bytes_
 
 
@@ -441,6 +443,8 @@ def main():
     dominant = max(kernel_times, key=lambda k: kernel_times[k][1])
     dom_ms = kernel_times[dominant][1] / max(1, kernel_times[dominant][0])
     if dominant == "expert_down_combine_gemm":
+        kf, kb = down_counts(cfg, touched, scatter_add=True)
+    elif dominant == "expert_down_gemm":
         kf, kb = down_counts(cfg, touched)
     else:
         kf, kb = gate_up_counts(cfg, touched)

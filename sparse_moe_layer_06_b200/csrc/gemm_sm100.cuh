@@ -7,7 +7,8 @@
 //                                      h[row, i]  = silu(clamp(G)) * clamp(U)
 //   EPI_DOWN_ATOMIC expert down+combine y[h, row] = sum_i Wd_e[i,h] * h_perm[row,i]
 //                                      out_acc[token(row), h] += w(row) * y
-//   EPI_DOWN_STORE  expert down        y_perm[row, h] = y
+//   EPI_DOWN_STORE  expert down        y_perm[row, h] = w(row) * y  (w = 1 when no
+//                                      routing weights are given)
 //
 // The weight matrix is always the MMA "A" operand (M = 128 weight rows per
 // tile) and the token rows are the "B" operand (N = 16..NMAX rows per tile,
@@ -149,7 +150,7 @@ struct GemmCfg {
     static constexpr int kBarrierBytes = 512;
     // (rounded to 128 bytes so that what follows stays 128-byte aligned)
     static constexpr int kSchedBytes = (5 * (kMaxSegments + 1) * 4 + 127) / 128 * 128;
-    static constexpr int kMetaBytes = (EPI == EPI_DOWN_ATOMIC) ? 2 * NMAX * 8 : 0;
+    static constexpr int kMetaBytes = kDown ? 2 * NMAX * 8 : 0;
     static constexpr int kEpiWarps = 8;
     static constexpr int kTailBytes = 1024 + kBarrierBytes + kSchedBytes + kMetaBytes;
     static constexpr int kMaxSmem = 227 * 1024;
@@ -436,7 +437,7 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
             if (!decode_tile(t, nblk, nseg, ss, args.special_seg, ti)) continue;
             int32_t* w_tok = reinterpret_cast<int32_t*>(s_meta) + mi * 2 * NMAX;
             float* w_wt = reinterpret_cast<float*>(w_tok + NMAX);
-            if constexpr (EPI == EPI_DOWN_ATOMIC) {
+            if constexpr (C::kDown) {
                 // token and routing weight of every column, fetched by the
                 // epilogue warps together before the accumulator is ready, so
                 // the loads overlap the main loop.  Two buffers alternate by
@@ -448,8 +449,8 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
                     int tok;
                     float wt;
                     if (r < args.routed_rows) {
-                        tok = __ldg(args.row_token + r);
-                        wt = __ldg(args.row_weight + r);
+                        tok = args.row_token ? __ldg(args.row_token + r) : r;
+                        wt = args.row_weight ? __ldg(args.row_weight + r) : 1.0f;
                     } else {
                         tok = r - args.routed_rows;
                         wt = 1.0f;
@@ -566,17 +567,39 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
                                     }
                                 }
                             }
+                        } else if (EPI == EPI_DOWN_STORE && !args.out_f32) {
+                            // weighted bf16 rows; lanes pair up (h, h+1) so each
+                            // store is a bf16x2 (H is even: lane pairs agree on m_ok)
+                            const bool odd = lane & 1;
+                            const int m_pair = m - (odd ? 1 : 0);
+                            __nv_bfloat16* yout = reinterpret_cast<__nv_bfloat16*>(args.out);
+#pragma unroll
+                            for (int j = 0; j < 16; j += 2) {
+                                const int c = c0 + j;
+                                const float a0 = v[j] * w_wt[c];
+                                const float a1 = v[j + 1] * w_wt[c + 1];
+                                const float mine = odd ? a1 : a0;
+                                const float send = odd ? a0 : a1;
+                                const float other = __shfl_xor_sync(0xffffffffu, send, 1);
+                                const int col = c + (odd ? 1 : 0);
+                                const __nv_bfloat162 pr = odd ? __floats2bfloat162_rn(other, mine)
+                                                              : __floats2bfloat162_rn(mine, other);
+                                if (m_ok && col < ti.n_valid) {
+                                    *reinterpret_cast<__nv_bfloat162*>(
+                                        yout + static_cast<size_t>(ti.out_row + col) * args.out_ld +
+                                        m_pair) = pr;
+                                }
+                            }
                         } else if (m_ok) {
 #pragma unroll
                             for (int j = 0; j < 16; ++j) {
                                 if (c0 + j < ti.n_valid) {
                                     const size_t o =
                                         static_cast<size_t>(ti.out_row + c0 + j) * args.out_ld + m;
-                                    if (EPI == EPI_LOGITS || args.out_f32) {
+                                    if constexpr (EPI == EPI_LOGITS) {
                                         reinterpret_cast<float*>(args.out)[o] = v[j];
                                     } else {
-                                        reinterpret_cast<__nv_bfloat16*>(args.out)[o] =
-                                            __float2bfloat16_rn(v[j]);
+                                        reinterpret_cast<float*>(args.out)[o] = v[j] * w_wt[c0 + j];
                                     }
                                 }
                             }

@@ -210,6 +210,18 @@ int pick_nmax(double mean_rows) {
     return 16;
 }
 
+// Token-row tile width of the down GEMM: the gate/up width (narrower tiles
+// re-read the weights more often, which costs power under the 1 kW cap more
+// than the double-buffered accumulator gains).  MOE_DOWN_NMAX overrides.
+int pick_down_nmax(int nmax_gu) {
+    static const int forced = [] {
+        const int v = env_int("MOE_DOWN_NMAX", 0);
+        return nmax_supported(v) ? v : 0;
+    }();
+    if (forced) return forced;
+    return nmax_gu;
+}
+
 // 128-row weight sub-tiles per down-projection tile: two, i.e. one 3D copy of
 // 32 KB of weights per pipeline stage against each token tile, which halves
 // the token-tile re-reads (the down GEMM is bound by the bulk-copy rows it
@@ -224,7 +236,13 @@ int pick_down_mb(int nmax) {
     return 2;
 }
 
-constexpr int kLogitsNmax = 64;
+// Router logits: 256 experts per tile (both 128-row blocks in one 256-row
+// box) against 32 tokens, so a 4096-token batch spreads over 128 CTAs.
+// MOE_LOGITS_NMAX=64 selects 64-token tiles.
+int logits_nmax() {
+    static const int v = env_int("MOE_LOGITS_NMAX", 32) == 64 ? 64 : 32;
+    return v;
+}
 constexpr int kLogitsMb = 2;
 
 // ------------------------------------------------------------------ workspace layout
@@ -240,7 +258,7 @@ struct Carve {
 
 struct Layout {
     size_t status, logits, idx, w, hist, base, counts, offsets, sched_gu, sched_dn, pos, src, row_w;
-    size_t x_perm, x_bf16, w_bf16, ws_bf16, h_perm, out_acc, y_bf16, total;
+    size_t x_perm, x_bf16, w_bf16, ws_bf16, h_perm, out_acc, y_perm, total;
 };
 
 int64_t perm_chunks(int64_t T) { return (T + kPermTokens - 1) / kPermTokens; }
@@ -290,7 +308,10 @@ Layout layout_for(const moe_problem* p, int call, int64_t ffn_rows = 0, int ffn_
             L.row_w = c.take(T * k * 4);
             L.x_perm = c.take(T * k * H * 2);
             L.h_perm = c.take(T * (k + S) * I * 2);
-            L.out_acc = c.take(T * H * 4);
+            // weighted expert rows (gather combine) or the fp32 token
+            // accumulator (scatter-add combine) share one region
+            L.out_acc = c.take(std::max(T * (k + S) * H * 2, T * H * 4));
+            L.y_perm = L.out_acc;
             if (f32) {
                 L.x_bf16 = c.take(T * H * 2);
                 L.w_bf16 = c.take(E * 3 * I * H * 2);
@@ -348,12 +369,14 @@ int32_t launch_gemm(int nmax, int mb, const GemmArgs& a, int64_t max_tiles, cuda
     int grid = static_cast<int>(std::min<int64_t>(sm_count(), std::max<int64_t>(1, max_tiles)));
     if constexpr (EPI == EPI_SWIGLU) {
         return launch_gemm_mb<EPI, 2>(nmax, a, grid, s, name);
-    } else if constexpr (EPI == EPI_DOWN_STORE) {
-        return launch_gemm_mb<EPI, 1>(nmax, a, grid, s, name);
     } else if constexpr (EPI == EPI_LOGITS) {
-        if (nmax != kLogitsNmax) return MOE_ERR_UNSUPPORTED;
-        if (mb == 2) return launch_gemm_n<EPI, kLogitsNmax, 2>(a, grid, s, name);
-        return launch_gemm_n<EPI, kLogitsNmax, 1>(a, grid, s, name);
+        if (nmax == 64) {
+            if (mb == 2) return launch_gemm_n<EPI, 64, 2>(a, grid, s, name);
+            return launch_gemm_n<EPI, 64, 1>(a, grid, s, name);
+        }
+        if (nmax != 32) return MOE_ERR_UNSUPPORTED;
+        if (mb == 2) return launch_gemm_n<EPI, 32, 2>(a, grid, s, name);
+        return launch_gemm_n<EPI, 32, 1>(a, grid, s, name);
     } else {
         if (mb == 2) return launch_gemm_mb<EPI, 2>(nmax, a, grid, s, name);
         return launch_gemm_mb<EPI, 1>(nmax, a, grid, s, name);
@@ -365,6 +388,19 @@ int32_t launch_gemm(int nmax, int mb, const GemmArgs& a, int64_t max_tiles, cuda
 int64_t max_tiles(int64_t rows_total, int nseg, int nmax, int64_t m_total,
                   int64_t rows_per_tile = 128) {
     return (rows_total / nmax + nseg) * ((m_total + rows_per_tile - 1) / rows_per_tile);
+}
+
+// How the expert rows are combined into token order (MOE_COMBINE=atomic picks
+// the fp32 scatter-add in the down GEMM's epilogue).  Default: the down
+// epilogue stores weighted bf16 rows and a gather kernel sums each token's
+// rows in slot order, which is deterministic and leaves the L2 atomic units
+// out of the critical path.
+bool combine_atomic() {
+    static const bool v = [] {
+        const char* e = std::getenv("MOE_COMBINE");
+        return e && std::strcmp(e, "atomic") == 0;
+    }();
+    return v;
 }
 
 // L2 cache hints on the GEMM operand loads (MOE_L2_HINTS=0 turns them off).
@@ -394,14 +430,14 @@ int32_t run_logits_bf16(const moe_problem* p, const void* x, const void* gate_w,
     for (int j = 0; j < kNumBoxSizes; ++j) a.tmB1[j] = a.tmB0[j];
     a.sched = nullptr;
     a.single_rows = static_cast<int32_t>(p->T);
-    a.single_chunk_len = kLogitsNmax;
+    const int lnmax = logits_nmax();
+    a.single_chunk_len = lnmax;
     a.nseg = 1;
     a.K = p->H;
     a.M_total = p->E;
     a.out = logits;
     a.out_ld = p->E;
-    return launch_gemm<EPI_LOGITS>(kLogitsNmax, mb, a,
-                                   max_tiles(p->T, 1, kLogitsNmax, p->E, 128 * mb), s,
+    return launch_gemm<EPI_LOGITS>(lnmax, mb, a, max_tiles(p->T, 1, lnmax, p->E, 128 * mb), s,
                                    "router_logits_gemm");
 }
 
@@ -448,9 +484,15 @@ __global__ void gather_kernel(const TIn* __restrict__ x, int64_t T, int H, int k
                               const int32_t* __restrict__ pos, int64_t n_rows,
                               TOut* __restrict__ x_perm, __nv_bfloat16* __restrict__ x_bf16,
                               float* __restrict__ acc_zero) {
+    // one warp per (token, segment of 32 * kBatch output vectors)
+    constexpr int kElems0 = 16 / sizeof(TOut);
+    constexpr int kSeg = 32 * 8;
     const int lane = threadIdx.x & 31;
-    const int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int nseg = (H / kElems0 + kSeg - 1) / kSeg;
+    const int64_t gw = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int64_t t = gw / nseg;
     if (t >= T) return;
+    const int seg = static_cast<int>(gw - t * nseg);
     int my_pos = -1;
     if (lane < k) {
         my_pos = pos[t * k + lane];
@@ -458,8 +500,10 @@ __global__ void gather_kernel(const TIn* __restrict__ x, int64_t T, int H, int k
     }
     constexpr int kElems = 16 / sizeof(TOut);  // elements per 16-byte output vector
     constexpr int kBatch = 8;  // 16-byte loads in flight per lane before the stores
+    static_assert(32 * kBatch == kSeg, "segment = one batch");
     const int nvec = H / kElems;
-    for (int v0 = 0; v0 < nvec; v0 += 32 * kBatch) {
+    {
+        const int v0 = seg * kSeg;
         uint4 packed[kBatch];
 #pragma unroll
         for (int b = 0; b < kBatch; ++b) {
@@ -498,8 +542,11 @@ __global__ void gather_kernel(const TIn* __restrict__ x, int64_t T, int H, int k
         }
     }
     if (acc_zero) {
+        // this segment's share of the token's fp32 accumulator row
+        const int per = (H / 4 + nseg - 1) / nseg;
         float4* z = reinterpret_cast<float4*>(acc_zero + t * H);
-        for (int v = lane; v < H / 4; v += 32) z[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int v = seg * per + lane; v < min(H / 4, (seg + 1) * per); v += 32)
+            z[v] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 }
 
@@ -509,7 +556,8 @@ template <typename TIn, typename TOut>
 int32_t run_gather(const TIn* x, int64_t T, int H, int k, const int32_t* pos, int64_t n_rows,
                    TOut* x_perm, __nv_bfloat16* x_bf16, float* acc_zero, cudaStream_t s) {
     const int warps = 8;
-    const unsigned blocks = static_cast<unsigned>((T + warps - 1) / warps);
+    const int64_t segs = (H / (16 / static_cast<int>(sizeof(TOut))) + 32 * 8 - 1) / (32 * 8);
+    const unsigned blocks = static_cast<unsigned>((T * segs + warps - 1) / warps);
     MOE_LAUNCH("dispatch_gather", s,
                gather_kernel<TIn, TOut><<<blocks, warps * 32, 0, s>>>(x, T, H, k, pos, n_rows,
                                                                       x_perm, x_bf16, acc_zero));
@@ -696,7 +744,8 @@ int32_t moe_grouped_swiglu_ffn(const moe_problem* p, const void* x_perm, int64_t
     }
     {
         GemmArgs a = base_args(status);
-        if (!make_tmap_down(&a.tmA0, wb, static_cast<int64_t>(n_groups) * 3 * I, H, 1))
+        const int mb = pick_down_mb(nmax);
+        if (!make_tmap_down(&a.tmA0, wb, static_cast<int64_t>(n_groups) * 3 * I, H, mb))
             return MOE_ERR_CUDA;
         if (!make_tmap_rows(a.tmB0, h, rows, I)) return MOE_ERR_CUDA;
         a.tmA1 = a.tmA0;
@@ -710,7 +759,8 @@ int32_t moe_grouped_swiglu_ffn(const moe_problem* p, const void* x_perm, int64_t
         a.out = y_perm;
         a.out_ld = static_cast<int32_t>(H);
         a.out_f32 = p->dtype == MOE_F32 ? 1 : 0;
-        MOE_TRY(launch_gemm<EPI_DOWN_STORE>(nmax, 1, a, max_tiles(rows, n_groups, nmax, H), s,
+        MOE_TRY(launch_gemm<EPI_DOWN_STORE>(nmax, mb, a,
+                                            max_tiles(rows, n_groups, nmax, H, 128 * mb), s,
                                             "expert_down_gemm"));
     }
     return MOE_OK;
@@ -785,18 +835,21 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
 
     // 2. dispatch bookkeeping + schedules
     const int nmax = pick_nmax(static_cast<double>(T * k) / E);
+    const int nmax_dn = pick_down_nmax(nmax);
     int32_t* sg = at<int32_t>(ws, L.sched_gu);
     int32_t* sd = at<int32_t>(ws, L.sched_dn);
     int32_t* pos = at<int32_t>(ws, L.pos);
     int32_t* src = at<int32_t>(ws, L.src);
     float* row_w = at<float>(ws, L.row_w);
     MOE_TRY(run_dispatch(p, idx, w, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base),
-                         at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets), sg, nmax, sd, nmax,
-                         pos, src, row_w, status, s));
+                         at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets), sg, nmax, sd,
+                         nmax_dn, pos, src, row_w, status, s));
 
     // 3. gather token rows (x -> x_perm), bf16 copy of x for fp32, zero accumulator
     __nv_bfloat16* x_perm = at<__nv_bfloat16>(ws, L.x_perm);
-    float* out_acc = at<float>(ws, L.out_acc);
+    const bool atomic_combine = combine_atomic();
+    float* out_acc = atomic_combine ? at<float>(ws, L.out_acc) : nullptr;
+    __nv_bfloat16* y_perm = at<__nv_bfloat16>(ws, L.y_perm);
     const void* x_b = x;
     if (f32) {
         MOE_TRY((run_gather<float, __nv_bfloat16>(static_cast<const float*>(x), T, p->H, p->top_k,
@@ -837,10 +890,12 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
         MOE_TRY(launch_gemm<EPI_SWIGLU>(nmax, 2, a, max_tiles(h_rows, nseg, nmax, I), s,
                                         "expert_gate_up_gemm"));
     }
-    // 5. grouped down GEMM, routing weight + scatter-add into the fp32 accumulator
+    // 5. grouped down GEMM; its epilogue applies the routing weight and either
+    //    stores the weighted rows (gather combine) or scatter-adds them into the
+    //    fp32 token accumulator
     {
         GemmArgs a = base_args(status);
-        const int mb = pick_down_mb(nmax);
+        const int mb = pick_down_mb(nmax_dn);
         if (!make_tmap_down(&a.tmA0, ew, E * 3 * I, H, mb)) return MOE_ERR_CUDA;
         if (!make_tmap_rows(a.tmB0, h, h_rows, I)) return MOE_ERR_CUDA;
         if (S) {
@@ -856,19 +911,44 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
         a.M_total = static_cast<int32_t>(H);
         a.a_seg_stride = static_cast<int32_t>(3 * I);
         a.a_off0 = static_cast<int32_t>(2 * I);
-        a.out = out_acc;
         a.out_ld = static_cast<int32_t>(H);
         a.n_tokens = static_cast<int32_t>(T);
         a.row_token = src;
         a.row_weight = row_w;
         a.routed_rows = static_cast<int32_t>(T * k);
-        MOE_TRY(launch_gemm<EPI_DOWN_ATOMIC>(nmax, mb, a,
-                                             max_tiles(h_rows, nseg, nmax, H, 128 * mb), s,
-                                             "expert_down_combine_gemm"));
+        const int64_t tiles = max_tiles(h_rows, nseg, nmax_dn, H, 128 * mb);
+        if (atomic_combine) {
+            a.out = out_acc;
+            MOE_TRY(launch_gemm<EPI_DOWN_ATOMIC>(nmax_dn, mb, a, tiles, s,
+                                                 "expert_down_combine_gemm"));
+        } else {
+            a.out = y_perm;
+            MOE_TRY(launch_gemm<EPI_DOWN_STORE>(nmax_dn, mb, a, tiles, s, "expert_down_gemm"));
+        }
     }
-    // 6. output cast
-    if (f32) return run_finalize<float>(out_acc, static_cast<float*>(out), T * H, s);
-    return run_finalize<__nv_bfloat16>(out_acc, static_cast<__nv_bfloat16*>(out), T * H, s);
+    // 6. token-order output
+    if (atomic_combine) {
+        if (f32) return run_finalize<float>(out_acc, static_cast<float*>(out), T * H, s);
+        return run_finalize<__nv_bfloat16>(out_acc, static_cast<__nv_bfloat16*>(out), T * H, s);
+    }
+    {
+        const int warps = 8;
+        const int64_t segs = (p->H / 8 + kSegVecs - 1) / kSegVecs;
+        const unsigned blocks = static_cast<unsigned>((T * segs + warps - 1) / warps);
+        const int64_t shared_row0 = S ? T * k : -1;
+        if (f32) {
+            MOE_LAUNCH("combine_gather", s,
+                       gather_sum_kernel<float><<<blocks, warps * 32, 0, s>>>(
+                           y_perm, pos, T, p->H, p->top_k, T * k, shared_row0,
+                           static_cast<float*>(out), status));
+        } else {
+            MOE_LAUNCH("combine_gather", s,
+                       gather_sum_kernel<__nv_bfloat16><<<blocks, warps * 32, 0, s>>>(
+                           y_perm, pos, T, p->H, p->top_k, T * k, shared_row0,
+                           static_cast<__nv_bfloat16*>(out), status));
+        }
+    }
+    return MOE_OK;
 }
 
 }  // extern "C"

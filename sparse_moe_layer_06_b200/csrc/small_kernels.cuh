@@ -389,6 +389,80 @@ __global__ void combine_kernel(const T* __restrict__ y_perm, const int32_t* __re
     }
 }
 
+// Fixed-order combine of weighted expert rows (the down GEMM already applied
+// the routing weights): out[t] = sum_j y[pos[t,j]] (j = 0..k-1 in slot order)
+// + y[shared_row0 + t] when shared_row0 >= 0, summed in fp32.  One warp per
+// (token, 512-value segment of H): 16-byte vectors, two per lane in flight per
+// row, so even a few tokens spread over many warps.
+constexpr int kSegVecs = 64;  // 16-byte vectors per warp segment
+
+template <typename TOut>
+__global__ void gather_sum_kernel(const __nv_bfloat16* __restrict__ y,
+                                  const int32_t* __restrict__ pos, int64_t T, int H, int k,
+                                  int64_t n_rows, int64_t shared_row0, TOut* __restrict__ out,
+                                  int32_t* status) {
+    const int lane = threadIdx.x & 31;
+    const int nvec = H / 8;
+    const int nseg = (nvec + kSegVecs - 1) / kSegVecs;
+    const int64_t gw = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int64_t t = gw / nseg;
+    if (t >= T) return;
+    const int seg = static_cast<int>(gw - t * nseg);
+    int my_pos = -1;
+    if (lane < k) {
+        const int p = pos[t * k + lane];
+        if (p < 0 || p >= n_rows) set_device_error(status, DEV_ERR_BAD_INDEX);
+        else my_pos = p;
+    }
+    const uint4* yv = reinterpret_cast<const uint4*>(y);
+    const int64_t row_vecs = nvec;
+    {
+        const int v0 = seg * kSegVecs;
+        const int va = v0 + lane, vb = v0 + 32 + lane;
+        const bool oka = va < nvec, okb = vb < nvec;
+        float acc_a[8], acc_b[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc_a[e] = acc_b[e] = 0.0f;
+        auto add8 = [](float (&acc)[8], const uint4& q) {
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(h2[e]);
+                acc[2 * e] += f.x;
+                acc[2 * e + 1] += f.y;
+            }
+        };
+#pragma unroll 4
+        for (int j = 0; j < k; ++j) {
+            const int r = __shfl_sync(0xffffffffu, my_pos, j);
+            if (r >= 0) {
+                if (oka) add8(acc_a, yv[r * row_vecs + va]);
+                if (okb) add8(acc_b, yv[r * row_vecs + vb]);
+            }
+        }
+        if (shared_row0 >= 0) {
+            const int64_t r = shared_row0 + t;
+            if (oka) add8(acc_a, yv[r * row_vecs + va]);
+            if (okb) add8(acc_b, yv[r * row_vecs + vb]);
+        }
+        auto put = [&](const float (&acc)[8], int v) {
+            if constexpr (sizeof(TOut) == 2) {
+                uint4 q;
+                __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&q);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) h2[e] = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
+                reinterpret_cast<uint4*>(out + t * H)[v] = q;
+            } else {
+                float4* o = reinterpret_cast<float4*>(out + t * H);
+                o[2 * v] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                o[2 * v + 1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+            }
+        };
+        if (oka) put(acc_a, va);
+        if (okb) put(acc_b, vb);
+    }
+}
+
 __global__ void cast_f32_bf16_kernel(const float* __restrict__ in, __nv_bfloat16* __restrict__ out,
                                      int64_t n) {
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
