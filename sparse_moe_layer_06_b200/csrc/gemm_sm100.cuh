@@ -107,13 +107,19 @@ struct GemmArgs {
     int32_t a_off1;        // unused (kept zero)
     void* out;
     int32_t out_ld;
-    int32_t n_tokens;          // EPI_DOWN_ATOMIC: rows of the accumulator
+    int32_t n_tokens;          // EPI_DOWN_ATOMIC: rows of the accumulator;
+                               // EPI_SWIGLU row gather: rows of gather_src
     const int32_t* row_token;  // EPI_DOWN_ATOMIC: token of each routed row
     const float* row_weight;   // EPI_DOWN_ATOMIC: routing weight of each routed row
     int32_t routed_rows;       // rows >= routed_rows belong to the shared expert
     float clip;                // EPI_SWIGLU clamp limit (+inf: none)
     int32_t out_f32;           // EPI_DOWN_STORE: fp32 (1) or bf16 (0) output
     int32_t l2_hints;          // 1: weights evict-first, token rows evict-last; 0: none
+    // EPI_SWIGLU row gather: when gather_tok != nullptr, ordinary segments
+    // take their token rows straight from gather_src ([n_tokens, K] bf16) at
+    // rows gather_tok[b_row + i] instead of from tmB0 (the permuted copy)
+    const int32_t* gather_tok;
+    const void* gather_src;
     int32_t* status;           // device error word
 };
 
@@ -152,7 +158,10 @@ struct GemmCfg {
     static constexpr int kSchedBytes = (5 * (kMaxSegments + 1) * 4 + 127) / 128 * 128;
     static constexpr int kMetaBytes = kDown ? 2 * NMAX * 8 : 0;
     static constexpr int kEpiWarps = 8;
-    static constexpr int kTailBytes = 1024 + kBarrierBytes + kSchedBytes + kMetaBytes;
+    // EPI_SWIGLU: token index of each row of the current tile (row gather)
+    static constexpr int kGatherBytes = kSwiGLU ? NMAX * 4 : 0;
+    static constexpr int kTailBytes =
+        1024 + kBarrierBytes + kSchedBytes + kMetaBytes + kGatherBytes;
     static constexpr int kMaxSmem = 227 * 1024;
     static constexpr int kStagesRaw = (kMaxSmem - kTailBytes) / kStageBytes;
     static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
@@ -209,6 +218,8 @@ __device__ __forceinline__ float fast_rcp(float d) {
     return r;
 }
 
+using bf16_raw_ptr = const __nv_bfloat16*;
+
 __device__ __forceinline__ float clamp_keep_nan(float v, float lim) {
     return v > lim ? lim : (v < -lim ? -lim : v);
 }
@@ -231,6 +242,7 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int32_t* s_sched = reinterpret_cast<int32_t*>(tail + C::kBarrierBytes);
     uint8_t* s_meta = tail + C::kBarrierBytes + C::kSchedBytes;
+    int32_t* s_gtok = reinterpret_cast<int32_t*>(s_meta + C::kMetaBytes);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -298,33 +310,65 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            const uint64_t pol_w =
-                args.l2_hints ? ptx::policy_evict_first() : ptx::policy_evict_normal();
-            const uint64_t pol_x =
-                args.l2_hints ? ptx::policy_evict_last() : ptx::policy_evict_normal();
-            uint32_t stage = 0, phase = 0;
-            uint32_t armed = 0, armed_phase = 0;  // per-stage bits
-            bool ok = true;
-            for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
-                TileInfo ti;
-                if (!decode_tile(t, nblk, nseg, ss, args.special_seg, ti)) continue;
-                const CUtensorMap* tA = ti.special ? &args.tmA1 : &args.tmA0;
-                const CUtensorMap* tB = ti.special ? args.tmB1 : args.tmB0;
-                const int a_base = ti.special ? 0 : ti.seg * args.a_seg_stride;
-                const uint32_t bytes = C::kABytes + ti.n_mma * 128;
-                for (int kb = 0; kb < ksteps; ++kb) {
-                    if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag)) {
-                        fail(DEV_ERR_TIMEOUT);
-                        ok = false;
-                        break;
+        // Lane 0 waits for free slots and issues the bulk tensor copies.  For
+        // a gathered tile (EPI_SWIGLU, ordinary segment, gather_tok set) the
+        // whole warp also copies the token rows from the unpermuted source
+        // with 16-byte cp.async: eight lanes per 128-byte row, written in the
+        // same 128-byte-swizzled layout a tensor copy produces.
+        const uint64_t pol_w =
+            args.l2_hints ? ptx::policy_evict_first() : ptx::policy_evict_normal();
+        const uint64_t pol_x =
+            args.l2_hints ? ptx::policy_evict_last() : ptx::policy_evict_normal();
+        const bf16_raw_ptr gsrc = reinterpret_cast<bf16_raw_ptr>(args.gather_src);
+        uint32_t stage = 0, phase = 0;
+        uint32_t armed = 0, armed_phase = 0;  // per-stage bits (lane 0)
+        bool ok = true;
+        for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
+            TileInfo ti;
+            if (!decode_tile(t, nblk, nseg, ss, args.special_seg, ti)) continue;
+            const CUtensorMap* tA = ti.special ? &args.tmA1 : &args.tmA0;
+            const CUtensorMap* tB = ti.special ? args.tmB1 : args.tmB0;
+            const int a_base = ti.special ? 0 : ti.seg * args.a_seg_stride;
+            const bool gather = C::kSwiGLU && args.gather_tok != nullptr && !ti.special;
+            if (gather) {
+                __syncwarp();  // the previous tile's rows are all issued
+                for (int i = lane; i < ti.n_mma; i += 32)
+                    s_gtok[i] = i < ti.n_valid ? __ldg(args.gather_tok + ti.b_row + i) : -1;
+                __syncwarp();
+            }
+            const uint32_t bytes = C::kABytes + (gather ? 0 : ti.n_mma * 128);
+            for (int kb = 0; kb < ksteps; ++kb) {
+                int got = 1;
+                if (lane == 0) got = ptx::mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag);
+                got = __shfl_sync(0xffffffffu, got, 0);
+                if (!got) {
+                    if (lane == 0) fail(DEV_ERR_TIMEOUT);
+                    ok = false;
+                    break;
+                }
+                uint8_t* sA = ring + stage * C::kStageBytes;
+                uint8_t* sB = sA + C::kABytes;
+                const int k0 = kb * 64;
+                if (gather) {
+                    const int chunk = lane & 7;
+                    for (int r = lane >> 3; r < ti.n_mma; r += 4) {
+                        int tok = s_gtok[r];
+                        if (static_cast<unsigned>(tok) >= static_cast<unsigned>(args.n_tokens))
+                            tok = -1;  // padding row, or an out-of-range index: zeros
+                        const void* src = tok >= 0
+                            ? static_cast<const void*>(gsrc + static_cast<size_t>(tok) * args.K +
+                                                       k0 + chunk * 8)
+                            : static_cast<const void*>(gsrc);
+                        ptx::cp_async_16(sB + r * 128 + ((chunk ^ (r & 7)) << 4), src,
+                                         tok >= 0 ? 16u : 0u);
                     }
-                    uint8_t* sA = ring + stage * C::kStageBytes;
-                    uint8_t* sB = sA + C::kABytes;
+                    ptx::cp_async_mbar_arrive(&full_bar[stage]);
+                    __syncwarp();  // every lane's arrival is counted before lane 0 arrives
+                }
+                if (lane == 0) {
                     ptx::mbar_arrive_expect_tx(&full_bar[stage], bytes);
                     armed |= 1u << stage;
                     armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
-                    const int k0 = kb * 64;
                     if constexpr (C::kDown) {
                         // MN-major A: one 3D copy of 2*MB chunks of 64 H-values
                         // x 64 K-rows, chunk-major in shared memory (8 KB each)
@@ -339,14 +383,10 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
                         ptx::tma_load_2d(sA, tA, k0, a_base + args.a_off0 + ti.blk * 256,
                                          &full_bar[stage], pol_w);
                     } else {
-#pragma unroll
-                        for (int j = 0; j < MB; ++j) {
-                            ptx::tma_load_2d(sA + j * C::kATileBytes, tA, k0,
-                                             a_base + args.a_off0 + (ti.blk * MB + j) * 128,
-                                             &full_bar[stage], pol_w);
-                        }
+                        ptx::tma_load_2d(sA, tA, k0, a_base + args.a_off0 + ti.blk * 128,
+                                         &full_bar[stage], pol_w);
                     }
-                    {
+                    if (!gather) {
                         int q = 0;
 #pragma unroll
                         for (int j = kNumBoxSizes - 1; j >= 0; --j) {
@@ -357,13 +397,17 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
                             }
                         }
                     }
-                    if (++stage == C::kStages) {
-                        stage = 0;
-                        phase ^= 1;
-                    }
+                }
+                if (++stage == C::kStages) {
+                    stage = 0;
+                    phase ^= 1;
                 }
             }
-            // never leave with bulk copies still writing into this CTA's smem
+        }
+        // never leave with copies still writing into this CTA's shared memory
+        ptx::cp_async_wait_all();
+        __syncwarp();
+        if (lane == 0) {
             for (int s = 0; s < C::kStages; ++s) {
                 if (armed & (1u << s)) {
                     ptx::mbar_wait(&full_bar[s], (armed_phase >> s) & 1u, nullptr);
@@ -392,6 +436,9 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
                         ok = false;
                         break;
                     }
+                    // token rows gathered with cp.async were written through
+                    // the generic proxy; the MMA reads them through the async one
+                    if constexpr (C::kSwiGLU) ptx::fence_proxy_async_smem();
                     ptx::tc_fence_after();
                     const uint32_t a_addr = ptx::smem_u32(ring + stage * C::kStageBytes);
                     const uint32_t b_addr = a_addr + C::kABytes;

@@ -325,3 +325,27 @@ def test_forward_repeatable_and_staged_path_agrees():
     ref = out1.float().cpu().numpy()
     assert_close_out(out_s.float().cpu().numpy(), ref.astype(np.float64), "staged vs fused",
                      tol=OUT_TOL)
+
+
+def test_forward_gather_variants_agree():
+    """The row gather inside the gate/up GEMM (MOE_FUSED_GATHER=1) and the
+    scatter-add combine (MOE_COMBINE=atomic) give the same layer: both are
+    checked against the oracle in a fresh process each."""
+    import os
+    import subprocess
+    import sys
+    code = (
+        "import torch, sys; sys.path.insert(0, '.'); sys.path.insert(0, 'tests');"
+        "from test_gpu_parity import cfg, run_forward;"
+        "from parity_util import forward_parity;"
+        "from sparse_moe_layer_06_b200.workloads import make_inputs;"
+        "c = cfg(T=300, H=512, E=16, k=4, I=384);"
+        "inp = make_inputs(c, seed=10, device='cuda');"
+        "out, idx, w = run_forward(c, inp);"
+        "forward_parity(inp, c, out, idx, w); print('ok')")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    for env in ({"MOE_FUSED_GATHER": "1"}, {"MOE_COMBINE": "atomic"},
+                {"MOE_FUSED_GATHER": "1", "MOE_COMBINE": "atomic"}):
+        r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True,
+                           text=True, env={**os.environ, **env}, timeout=600)
+        assert r.returncode == 0 and "ok" in r.stdout, (env, r.stdout[-2000:], r.stderr[-2000:])
