@@ -57,6 +57,9 @@ def _load():
             lib.oracle_expert_rows.argtypes = [I32, I32, I32, I32, P, P, P, D, P, P, I64, P]
             lib.oracle_permute.argtypes = [I64, I32, I32, P, P, P, P, P]
             lib.oracle_combine.argtypes = [I64, I32, I32, P, P, P, P, P]
+            lib.oracle_router_stats.argtypes = [I64, I32, I32, I32, I32, P, P, P, D, P, P, P, P,
+                                                P, P]
+            lib.oracle_router_stats.restype = None
             lib.oracle_num_threads.restype = ctypes.c_int
             for f in (lib.oracle_route, lib.oracle_forward, lib.oracle_dense_bruteforce,
                       lib.oracle_expert_rows, lib.oracle_permute, lib.oracle_combine):
@@ -226,6 +229,29 @@ def combine(y_perm, pos, w, shared_y=None):
     _load().oracle_combine(T, H, k, ya.ctypes.data, pa.ctypes.data, wa.ctypes.data, sp,
                            out.ctypes.data)
     return out
+
+
+def router_stats(x, gate_w, top_k: int, logit_bias=None, momentum: float = 0.9,
+                 ema_counts=None, ema_total=None):
+    """Load-balancing statistics over all tokens: dict(P [E], f [E], counts [E]
+    int64, aux float, ema_counts [E] or None, ema_total float or None)."""
+    T, H = x.shape
+    E = gate_w.shape[0]
+    xa, xp, dt = _stored(x)
+    ga, gp, _ = _stored(gate_w)
+    ba, bp = _f32(logit_bias)
+    P = np.zeros(E, np.float64)
+    f = np.zeros(E, np.float64)
+    cnt = np.zeros(E, np.int64)
+    aux = np.zeros(1, np.float64)
+    ec = None if ema_counts is None else np.array(ema_counts, dtype=np.float64, copy=True)
+    et = None if ema_total is None else np.array([ema_total], dtype=np.float64)
+    _load().oracle_router_stats(T, H, E, top_k, dt, xp, gp, bp, float(momentum), P.ctypes.data,
+                                f.ctypes.data, cnt.ctypes.data, aux.ctypes.data,
+                                None if ec is None else ec.ctypes.data,
+                                None if et is None else et.ctypes.data)
+    return dict(P=P, f=f, counts=cnt, aux=float(aux[0]), ema_counts=ec,
+                ema_total=None if et is None else float(et[0]))
 
 
 def near_tie_alternatives(probs_row: np.ndarray, k: int, rel: float = 1e-5):

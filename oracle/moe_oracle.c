@@ -355,6 +355,53 @@ void oracle_combine(int64_t T, int H, int k, const double* y_perm,
     }
 }
 
+/*
+ * oracle_router_stats: the router's load-balancing statistics (page
+ * "腾讯混元Hy3正式版深度解析", SparseMoERouter._compute_load_balancing_loss and
+ * the expert-count update in forward), over all T tokens:
+ *   P[e]   = (1/T) * sum_t p[t,e]                 mean routing probability
+ *   cnt[e] = #{(t,j) : idx[t,j] == e}             selections of expert e
+ *   f[e]   = cnt[e] / (T*k)                        selection frequency
+ *   aux    = E * sum_e P[e] * f[e]                 auxiliary loss
+ *   ema_counts[e] <- momentum * ema_counts[e] + (1 - momentum) * cnt[e]
+ *   ema_total     <- momentum * ema_total + (1 - momentum) * T
+ * (the sketch uses momentum 0.9).  p and idx are steps 2 and 3 above.
+ * ema_counts / ema_total may be NULL (not updated).
+ */
+void oracle_router_stats(int64_t T, int H, int E, int k, int dtype, const void* x,
+                         const void* gate_w, const float* bias, double momentum, double* P,
+                         double* f, int64_t* cnt, double* aux, double* ema_counts,
+                         double* ema_total) {
+    for (int e = 0; e < E; ++e) {
+        P[e] = 0.0;
+        cnt[e] = 0;
+    }
+    double* l = (double*)malloc(sizeof(double) * (size_t)E);
+    double* p = (double*)malloc(sizeof(double) * (size_t)E);
+    int32_t* idx = (int32_t*)malloc(sizeof(int32_t) * (size_t)k);
+    double* w = (double*)malloc(sizeof(double) * (size_t)k);
+    for (int64_t t = 0; t < T; ++t) {
+        route_one(t, H, E, k, dtype, x, gate_w, bias, 1.0, l, p, idx, w);
+        for (int e = 0; e < E; ++e) P[e] += p[e];
+        for (int j = 0; j < k; ++j) cnt[idx[j]] += 1;
+    }
+    double a = 0.0;
+    for (int e = 0; e < E; ++e) {
+        P[e] /= (double)T;
+        f[e] = (double)cnt[e] / ((double)T * (double)k);
+        a += P[e] * f[e];
+    }
+    *aux = (double)E * a;
+    if (ema_counts)
+        for (int e = 0; e < E; ++e)
+            ema_counts[e] = momentum * ema_counts[e] + (1.0 - momentum) * (double)cnt[e];
+    if (ema_total) *ema_total = momentum * (*ema_total) + (1.0 - momentum) * (double)T;
+    free(l);
+    free(p);
+    free(idx);
+    free(w);
+}
+
 /* Number of OpenMP threads the oracle will use (for reporting). */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

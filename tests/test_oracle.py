@@ -329,3 +329,57 @@ def test_hy4_config_matches_printed_hyperparameters():
     assert 0.9 * g["total_params"] < experts_total < g["total_params"]
     assert experts_active < g["activated_params"]
     assert g["moe_layers"] + g["dense_layers"] == g["num_hidden_layers"]
+
+
+# ---------------------------------------------------------------- router statistics pins
+
+def test_router_stats_uniform_router_closed_form():
+    # all-zero gate: every probability is 1/E, ties pick experts 0..k-1 for
+    # every token, so P = 1/E, f = 1/k on the first k experts, aux = 1
+    E, k, T = 8, 3, 10
+    x = torch.randn(T, 64, generator=torch.Generator().manual_seed(0))
+    g = torch.zeros(E, 64)
+    st = oracle.router_stats(x, g, k)
+    np.testing.assert_allclose(st["P"], 1.0 / E, rtol=1e-15)
+    np.testing.assert_array_equal(st["counts"], [T] * k + [0] * (E - k))
+    assert st["aux"] == pytest.approx(1.0, rel=1e-15)
+
+
+def test_router_stats_two_token_hand_example():
+    # E=2, k=1, one-hot tokens: logits (2, 0) and (0, 1)
+    x = torch.zeros(2, 64)
+    x[0, 0] = 1.0
+    x[1, 1] = 1.0
+    g = torch.zeros(2, 64)
+    g[0, 0] = 2.0
+    g[1, 1] = 1.0
+    st = oracle.router_stats(x, g, 1)
+    p0 = [math.exp(2) / (math.exp(2) + 1), 1 / (math.exp(2) + 1)]
+    p1 = [1 / (1 + math.e), math.e / (1 + math.e)]
+    P = [(p0[0] + p1[0]) / 2, (p0[1] + p1[1]) / 2]
+    np.testing.assert_allclose(st["P"], P, rtol=1e-14)
+    np.testing.assert_array_equal(st["counts"], [1, 1])
+    assert st["aux"] == pytest.approx(2 * (P[0] * 0.5 + P[1] * 0.5), rel=1e-14)
+
+
+def test_router_stats_match_torch_composition_and_ema_closed_form():
+    cfg = small_cfg(E=16, k=4, T=64)
+    inp = make_inputs(cfg, seed=21)
+    st = oracle.router_stats(inp["x"], inp["gate_w"], cfg.top_k)
+    logits = f64(inp["x"]) @ f64(inp["gate_w"]).T
+    p = torch.softmax(logits, -1)
+    _, ti = torch.topk(p, cfg.top_k, -1)
+    counts = torch.bincount(ti.reshape(-1), minlength=cfg.E).numpy()
+    np.testing.assert_allclose(st["P"], p.mean(0).numpy(), rtol=1e-13)
+    np.testing.assert_array_equal(st["counts"], counts)
+    assert st["aux"] == pytest.approx(cfg.E * float((p.mean(0).numpy() * counts).sum())
+                                      / (cfg.T * cfg.top_k), rel=1e-13)
+    # EMA after n identical steps: c_n = m^n c_0 + (1 - m^n) counts
+    m, c0 = 0.9, np.linspace(0.0, 5.0, cfg.E)
+    ema, tot = c0.copy(), 3.0
+    for _ in range(5):
+        s2 = oracle.router_stats(inp["x"], inp["gate_w"], cfg.top_k, ema_counts=ema,
+                                 ema_total=tot, momentum=m)
+        ema, tot = s2["ema_counts"], s2["ema_total"]
+    np.testing.assert_allclose(ema, m ** 5 * c0 + (1 - m ** 5) * counts, rtol=1e-12)
+    assert tot == pytest.approx(m ** 5 * 3.0 + (1 - m ** 5) * cfg.T, rel=1e-13)
