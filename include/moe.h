@@ -69,7 +69,8 @@ typedef enum {
     MOE_CALL_PERMUTE = 2,
     MOE_CALL_FFN = 3,
     MOE_CALL_COMBINE = 4,
-    MOE_CALL_FORWARD = 5
+    MOE_CALL_FORWARD = 5,
+    MOE_CALL_ROUTER_STATS = 6
 } moe_call;
 
 typedef struct {
@@ -218,6 +219,24 @@ int32_t moe_forward(const moe_problem* problem, const void* x, const void* gate_
 int32_t moe_route_noalloc(const moe_problem* problem, const void* x, const void* gate_w,
                           const float* logit_bias, int32_t* topk_idx, float* topk_w,
                           void* stream);
+
+/*
+ * moe_router_stats -- the router's load-balancing statistics over the T
+ * tokens (page "腾讯混元Hy3正式版深度解析", SparseMoERouter: the auxiliary
+ * load-balancing loss and the running expert counts):
+ *   P_out[e]  = (1/T) sum_t softmax(logits[t] + bias)[e]   mean probability  [E] fp32
+ *   f_out[e]  = #{(t,j): topk_idx[t,j] == e} / (T*top_k)   selection share   [E] fp32
+ *   aux_out[0] = E * sum_e P_out[e] * f_out[e]             auxiliary loss    [1] fp32
+ *   ema_counts[e] <- m*ema_counts[e] + (1-m)*count[e]      [E] fp32 in/out, or NULL
+ *   ema_total[0]  <- m*ema_total[0] + (1-m)*T              [1] fp32 in/out, or NULL
+ * with m = momentum in [0,1] (the sketch uses 0.9); all pointers are device
+ * memory.  The routing (logits, top-k) is the one moe_route computes.  Sums
+ * are taken in a fixed order, so the results are reproducible.  T must be >= 1.
+ */
+int32_t moe_router_stats(const moe_problem* problem, const void* x, const void* gate_w,
+                         const float* logit_bias, float* P_out, float* f_out, float* aux_out,
+                         float* ema_counts, float* ema_total, float momentum, void* workspace,
+                         size_t ws_bytes, void* stream);
 
 /* Copy the device error word of `workspace` to *status_out (host), waiting
  * for the stream.  Returns MOE_OK or MOE_ERR_CUDA / MOE_ERR_INVALID_ARG. */

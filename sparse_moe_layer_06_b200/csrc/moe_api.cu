@@ -257,7 +257,7 @@ struct Carve {
 };
 
 struct Layout {
-    size_t status, logits, idx, w, hist, base, counts, offsets, sched_gu, sched_dn, pos, src, row_w;
+    size_t status, logits, idx, w, hist, base, counts, offsets, partial, sched_gu, sched_dn, pos, src, row_w;
     size_t x_perm, x_bf16, w_bf16, ws_bf16, h_perm, out_acc, y_perm, total;
 };
 
@@ -291,6 +291,13 @@ Layout layout_for(const moe_problem* p, int call, int64_t ffn_rows = 0, int ffn_
             }
             break;
         case MOE_CALL_COMBINE:
+            break;
+        case MOE_CALL_ROUTER_STATS:
+            L.logits = c.take(T * E * 4);
+            L.idx = c.take(T * k * 4);
+            L.w = c.take(T * k * 4);
+            L.partial = c.take(((T + kStatsTokensPerBlock - 1) / kStatsTokensPerBlock) * E * 4);
+            L.counts = c.take(E * 4);
             break;
         case MOE_CALL_FORWARD:
         default:
@@ -632,7 +639,7 @@ const char* moe_status_string(int32_t status) {
 
 size_t moe_workspace_size(const moe_problem* p, int32_t call) {
     if (check_problem(p) != MOE_OK) return 0;
-    if (call < MOE_CALL_ROUTE || call > MOE_CALL_FORWARD) return 0;
+    if (call < MOE_CALL_ROUTE || call > MOE_CALL_ROUTER_STATS) return 0;
     if (call == MOE_CALL_FFN) {
         // the FFN workspace depends on rows/groups; size it for the routed
         // rows of this problem (T*top_k) and E groups, the larger of the two
@@ -1022,6 +1029,37 @@ int32_t moe_route_noalloc(const moe_problem* p, const void* x, const void* gate_
     if (cudaMemsetAsync(status, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
     MOE_TRY(run_logits(p, x, gate_w, logits, status, s));
     return run_topk(p, logits, bias, topk_idx, topk_w, s);
+}
+
+int32_t moe_router_stats(const moe_problem* p, const void* x, const void* gate_w,
+                         const float* bias, float* P_out, float* f_out, float* aux_out,
+                         float* ema_counts, float* ema_total, float momentum, void* ws,
+                         size_t ws_bytes, void* stream) {
+    MOE_TRY(check_problem(p));
+    if (!x || !gate_w || !P_out || !f_out || !aux_out || !ws) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(gate_w) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+    if (!(momentum >= 0.0f && momentum <= 1.0f)) return MOE_ERR_INVALID_ARG;
+    if (p->T == 0) return MOE_ERR_INVALID_ARG;  // a mean over no tokens is undefined
+    const Layout L = layout_for(p, MOE_CALL_ROUTER_STATS);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t* status = at<int32_t>(ws, L.status);
+    float* logits = at<float>(ws, L.logits);
+    int32_t* idx = at<int32_t>(ws, L.idx);
+    int32_t* counts = at<int32_t>(ws, L.counts);
+    float* partial = at<float>(ws, L.partial);
+    MOE_TRY(run_logits(p, x, gate_w, logits, status, s));
+    MOE_TRY(run_topk(p, logits, bias, idx, at<float>(ws, L.w), s));
+    if (cudaMemsetAsync(counts, 0, p->E * sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+    const int nblocks = static_cast<int>((p->T + kStatsTokensPerBlock - 1) / kStatsTokensPerBlock);
+    MOE_LAUNCH("router_prob_partial", s,
+               router_prob_partial_kernel<<<nblocks, 256, 0, s>>>(logits, bias, idx, p->T, p->E,
+                                                                  p->top_k, partial, counts));
+    MOE_LAUNCH("router_stats_final", s,
+               router_stats_final_kernel<<<1, kMaxExperts, 0, s>>>(
+                   partial, nblocks, counts, p->T, p->E, p->top_k, momentum, P_out, f_out,
+                   aux_out, ema_counts, ema_total));
+    return MOE_OK;
 }
 
 int32_t moe_read_device_status(const void* ws, int32_t* status_out, void* stream) {

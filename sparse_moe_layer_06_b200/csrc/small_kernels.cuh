@@ -109,6 +109,102 @@ __global__ void topk_kernel(const float* __restrict__ logits, const float* __res
     }
 }
 
+// ------------------------------------------------------------------ router statistics
+
+constexpr int kStatsTokensPerBlock = 64;  // 8 warps x 8 tokens
+
+// Per-block sums of the routing probabilities p[t,e] = softmax(logits[t] + bias)
+// over a fixed block of 64 tokens, in a fixed order (warp w sums its 8 tokens
+// in turn, then the 8 warp sums are added in warp order); also counts the
+// selected experts into `counts` (integer atomics: order-independent).
+__global__ void router_prob_partial_kernel(const float* __restrict__ logits,
+                                           const float* __restrict__ bias,
+                                           const int32_t* __restrict__ idx, int64_t T, int E,
+                                           int k, float* __restrict__ partial,
+                                           int32_t* __restrict__ counts) {
+    __shared__ float s_sum[8][kMaxExperts];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int kPer = kMaxExperts / 32;
+    float acc[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) acc[i] = 0.0f;
+    for (int q = 0; q < kStatsTokensPerBlock / 8; ++q) {
+        const int64_t t = static_cast<int64_t>(blockIdx.x) * kStatsTokensPerBlock + warp * 8 + q;
+        if (t >= T) break;
+        float v[kPer];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int e = lane + 32 * i;
+            v[i] = -INFINITY;
+            if (e < E) {
+                v[i] = logits[t * E + e] + (bias ? bias[e] : 0.0f);
+                mx = fmaxf(mx, v[i]);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        float z = 0.0f;
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            v[i] = (lane + 32 * i < E) ? expf(v[i] - mx) : 0.0f;
+            z += v[i];
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) acc[i] += v[i] / z;
+        if (lane < k) {
+            const int e = idx[t * k + lane];
+            if (e >= 0 && e < E) atomicAdd(&counts[e], 1);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) s_sum[warp][lane + 32 * i] = acc[i];
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        float s = 0.0f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) s += s_sum[w][e];
+        partial[static_cast<size_t>(blockIdx.x) * E + e] = s;
+    }
+}
+
+// One CTA: P = sum of the per-block sums (in block order, fp64) / T,
+// f = counts / (T k), aux = E * sum_e P_e f_e (fixed-order reduction), and the
+// moving averages ema_counts = m * ema_counts + (1 - m) * counts,
+// ema_total = m * ema_total + (1 - m) * T.
+__global__ void router_stats_final_kernel(const float* __restrict__ partial, int nblocks,
+                                          const int32_t* __restrict__ counts, int64_t T, int E,
+                                          int k, float momentum, float* __restrict__ P_out,
+                                          float* __restrict__ f_out, float* __restrict__ aux_out,
+                                          float* ema_counts, float* ema_total) {
+    __shared__ double s_prod[kMaxExperts];
+    const int e = threadIdx.x;
+    double prod = 0.0;
+    if (e < E) {
+        double sum = 0.0;
+        for (int b = 0; b < nblocks; ++b) sum += partial[static_cast<size_t>(b) * E + e];
+        const double P = sum / static_cast<double>(T);
+        const double f = static_cast<double>(counts[e]) / (static_cast<double>(T) * k);
+        P_out[e] = static_cast<float>(P);
+        f_out[e] = static_cast<float>(f);
+        prod = P * f;
+        if (ema_counts)
+            ema_counts[e] = momentum * ema_counts[e] + (1.0f - momentum) * counts[e];
+    }
+    s_prod[e] = prod;
+    __syncthreads();
+    for (int s = kMaxExperts / 2; s > 0; s >>= 1) {
+        if (e < s) s_prod[e] += s_prod[e + s];
+        __syncthreads();
+    }
+    if (e == 0) {
+        *aux_out = static_cast<float>(E * s_prod[0]);
+        if (ema_total) *ema_total = momentum * (*ema_total) + (1.0f - momentum) * T;
+    }
+}
+
 // ------------------------------------------------------------------ dispatch
 
 // Build, for the warp's 32 tokens, one bit mask per expert of the lanes whose

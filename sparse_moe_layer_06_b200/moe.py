@@ -25,13 +25,13 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE = 0, 1, 2, 3
 MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_BAD_INDEX = 4, 5, 6
 MOE_F32, MOE_BF16 = 0, 1
 (MOE_CALL_ROUTE, MOE_CALL_ROUTER_LOGITS, MOE_CALL_PERMUTE, MOE_CALL_FFN, MOE_CALL_COMBINE,
- MOE_CALL_FORWARD) = range(6)
+ MOE_CALL_FORWARD, MOE_CALL_ROUTER_STATS) = range(7)
 
 EXPORTED = (
     "moe_workspace_size", "moe_status_string", "moe_router_logits", "moe_route", "moe_permute",
     "moe_grouped_swiglu_ffn", "moe_combine", "moe_forward", "moe_read_device_status",
     "moe_clear_device_status", "moe_launch_count", "moe_profile_start", "moe_profile_stop",
-    "moe_route_noalloc",
+    "moe_route_noalloc", "moe_router_stats",
 )
 ROUTE_NOALLOC_SCRATCH_BYTES = 1 << 20
 
@@ -112,6 +112,7 @@ def load_library(path: str = LIB_PATH):
             "moe_profile_start": (I32, [I32]),
             "moe_profile_stop": (I32, [ctypes.POINTER(KernelTimeC), I32, ctypes.POINTER(I32)]),
             "moe_route_noalloc": (I32, [PP, P, P, P, P, P, P]),
+            "moe_router_stats": (I32, [PP, P, P, P, P, P, P, P, P, ctypes.c_float, P, SZ, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -194,6 +195,20 @@ def moe_route_noalloc(problem, x, gate_w, logit_bias, topk_idx, topk_w, stream=N
         _ptr(logit_bias, torch.float32, "logit_bias", optional=True),
         _ptr(topk_idx, torch.int32, "topk_idx"), _ptr(topk_w, torch.float32, "topk_w"),
         _stream(stream)), "moe_route_noalloc")
+
+
+def moe_router_stats(problem, x, gate_w, logit_bias, P_out, f_out, aux_out, ema_counts,
+                     ema_total, momentum, workspace, stream=None):
+    pc = problem.c()
+    _check(load_library().moe_router_stats(
+        ctypes.byref(pc), _ptr(x, problem.dtype, "x"), _ptr(gate_w, problem.dtype, "gate_w"),
+        _ptr(logit_bias, torch.float32, "logit_bias", optional=True),
+        _ptr(P_out, torch.float32, "P_out"), _ptr(f_out, torch.float32, "f_out"),
+        _ptr(aux_out, torch.float32, "aux_out"),
+        _ptr(ema_counts, torch.float32, "ema_counts", optional=True),
+        _ptr(ema_total, torch.float32, "ema_total", optional=True), float(momentum),
+        _ptr(workspace, None, "workspace"), workspace.numel(), _stream(stream)),
+        "moe_router_stats")
 
 
 def moe_permute(problem, topk_idx, x, offsets, pos, src_token, x_perm, workspace, stream=None):
