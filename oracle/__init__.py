@@ -60,6 +60,17 @@ def _load():
             lib.oracle_router_stats.argtypes = [I64, I32, I32, I32, I32, P, P, P, D, P, P, P, P,
                                                 P, P]
             lib.oracle_router_stats.restype = None
+            lib.e4m3_decode.argtypes = [ctypes.c_uint8]
+            lib.e4m3_decode.restype = ctypes.c_double
+            lib.e4m3_encode.argtypes = [ctypes.c_double]
+            lib.e4m3_encode.restype = ctypes.c_uint8
+            lib.pow2_scale.argtypes = [ctypes.c_double]
+            lib.pow2_scale.restype = ctypes.c_double
+            lib.oracle_quantize_weights_fp8.argtypes = [I32, I32, I32, I32, P, P, P, P]
+            lib.oracle_quantize_weights_fp8.restype = None
+            lib.oracle_forward_fp8.argtypes = [I64, I32, I32, I32, I32, I32, P, P, P, P, P, P, P,
+                                               P, P, D, D, P, I64, P, P, P, P]
+            lib.oracle_forward_fp8.restype = None
             lib.oracle_num_threads.restype = ctypes.c_int
             for f in (lib.oracle_route, lib.oracle_forward, lib.oracle_dense_bruteforce,
                       lib.oracle_expert_rows, lib.oracle_permute, lib.oracle_combine):
@@ -252,6 +263,68 @@ def router_stats(x, gate_w, top_k: int, logit_bias=None, momentum: float = 0.9,
                                 None if et is None else et.ctypes.data)
     return dict(P=P, f=f, counts=cnt, aux=float(aux[0]), ema_counts=ec,
                 ema_total=None if et is None else float(et[0]))
+
+
+def e4m3_decode(code: int) -> float:
+    return float(_load().e4m3_decode(int(code) & 0xFF))
+
+
+def e4m3_encode(v: float) -> int:
+    return int(_load().e4m3_encode(float(v)))
+
+
+def pow2_scale(amax: float) -> float:
+    return float(_load().pow2_scale(float(amax)))
+
+
+def quantize_weights_fp8(expert_w):
+    """[E,3,I,H] weights -> (codes uint8 [E,3,I,H], gate/up row scales [E,2,I]
+    f64, down column scales [E,H] f64)."""
+    E, three, I, H = expert_w.shape
+    wa, wp, dt = _stored(expert_w)
+    q = np.zeros((E, 3, I, H), np.uint8)
+    s_gu = np.zeros((E, 2, I), np.float64)
+    s_d = np.zeros((E, H), np.float64)
+    _load().oracle_quantize_weights_fp8(E, I, H, dt, wp, q.ctypes.data, s_gu.ctypes.data,
+                                        s_d.ctypes.data)
+    return q, s_gu, s_d
+
+
+def forward_fp8(x, gate_w, q, s_gu, s_d, shared_q, shared_s_gu, shared_s_d, top_k: int,
+                scale: float, clip: float, logit_bias=None, tokens=None, forced_idx=None):
+    """Layer forward with FP8 expert weights (see moe_oracle.c).  q/s_gu/s_d as
+    returned by quantize_weights_fp8; shared_* for one shared expert or None."""
+    T, H = x.shape
+    E = q.shape[0]
+    I = q.shape[2]
+    xa, xp, dt = _stored(x)
+    ga, gp, _ = _stored(gate_w)
+    ba, bp = _f32(logit_bias)
+    qa = np.ascontiguousarray(q, dtype=np.uint8)
+    sg = np.ascontiguousarray(s_gu, dtype=np.float64)
+    sd = np.ascontiguousarray(s_d, dtype=np.float64)
+    if shared_q is not None:
+        sqa = np.ascontiguousarray(shared_q, dtype=np.uint8)
+        ssg = np.ascontiguousarray(shared_s_gu, dtype=np.float64)
+        ssd = np.ascontiguousarray(shared_s_d, dtype=np.float64)
+        sq_p, ssg_p, ssd_p = sqa.ctypes.data, ssg.ctypes.data, ssd.ctypes.data
+    else:
+        sq_p = ssg_p = ssd_p = None
+    tok = _tokens(T, tokens)
+    n = tok.size
+    fp = None
+    if forced_idx is not None:
+        fa = np.ascontiguousarray(np.asarray(forced_idx, dtype=np.int32).reshape(n, top_k))
+        fp = fa.ctypes.data
+    out = np.zeros((n, H), np.float64)
+    idx = np.zeros((n, top_k), np.int32)
+    w = np.zeros((n, top_k), np.float64)
+    if n:
+        _load().oracle_forward_fp8(T, H, E, top_k, I, dt, xp, gp, bp, qa.ctypes.data,
+                                   sg.ctypes.data, sd.ctypes.data, sq_p, ssg_p, ssd_p,
+                                   float(scale), float(clip), tok.ctypes.data, n, fp,
+                                   out.ctypes.data, idx.ctypes.data, w.ctypes.data)
+    return dict(out=out, idx=idx, w=w)
 
 
 def near_tie_alternatives(probs_row: np.ndarray, k: int, rel: float = 1e-5):

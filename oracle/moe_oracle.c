@@ -402,6 +402,191 @@ void oracle_router_stats(int64_t T, int H, int E, int k, int dtype, const void* 
     free(w);
 }
 
+/* ------------------------------------------------------------------------
+ * FP8 expert weights (the FP8 deployment noted on page "1M上下文实战：Hy4
+ * preview如何从容处理百万token级长文档", section "最快部署 1M 上下文"; the pages
+ * give no number format, so the reading is stated here).
+ *
+ * E4M3 (OCP FP8): 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits; no
+ * infinities; code S.1111.111 is NaN; largest finite 448; subnormals
+ * m * 2^-9.  Encoding rounds to nearest, ties to even, saturating to +-448.
+ *
+ * Scales are powers of two, so dividing by a scale is exact in any binary
+ * floating-point format and the encoding decision is the same wherever it
+ * is taken:
+ *   pow2_scale(amax) = 2^ceil(log2(amax / 448))  (1 when amax == 0)
+ * Weights: gate/up rows i and down columns h each get
+ *   s = pow2_scale(max |w| over that row / column), q = e4m3(w / s).
+ * Token rows x_t: s_x = pow2_scale(max_h |x_t[h]|), q = e4m3(x_t / s_x).
+ * The SwiGLU output h is bounded by the clamp L (|h| <= silu(L) L), so it
+ * uses one fixed scale s_h = pow2_scale(silu(L) * L): h_q = e4m3(h / s_h).
+ * The expert FFN then computes, in fp64 on the decoded codes,
+ *   g[i] = s_x s_g[i] sum_h xq[h] gq[i,h],   u[i] likewise,
+ *   h[i] = silu(clamp g) clamp u,   y[c] = s_h s_d[c] sum_i hq[i] dq[i,c].
+ * ------------------------------------------------------------------------ */
+
+double e4m3_decode(uint8_t code) {
+    const int sign = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+uint8_t e4m3_encode(double v) {
+    if (isnan(v)) return 0x7F;
+    const int sign = v < 0 || (v == 0.0 && signbit(v));
+    double a = fabs(v);
+    if (a >= 448.0) return (uint8_t)((sign << 7) | 0x7E);
+    /* all finite codes in increasing order of magnitude: pick the nearest,
+     * ties to the even code (codes 0..126 encode increasing magnitudes) */
+    int lo = 0, hi = 126;
+    while (hi - lo > 1) {
+        int mid = (lo + hi) / 2;
+        if (e4m3_decode((uint8_t)mid) <= a) lo = mid;
+        else hi = mid;
+    }
+    double dlo = a - e4m3_decode((uint8_t)lo), dhi = e4m3_decode((uint8_t)hi) - a;
+    int c;
+    if (dlo < dhi) c = lo;
+    else if (dhi < dlo) c = hi;
+    else c = (lo % 2 == 0) ? lo : hi;
+    return (uint8_t)((sign << 7) | c);
+}
+
+double pow2_scale(double amax) {
+    if (!(amax > 0.0)) return 1.0;
+    return ldexp(1.0, (int)ceil(log2(amax / 448.0)));
+}
+
+/*
+ * oracle_quantize_weights_fp8: w [n_mats/3 experts,3,I,H] (bf16/fp32) ->
+ * q (same shape, E4M3 codes), s_gu [n_experts,2,I] (gate, up row scales),
+ * s_d [n_experts,H] (down column scales).
+ */
+void oracle_quantize_weights_fp8(int n_experts, int I, int H, int dtype, const void* w,
+                                 uint8_t* q, double* s_gu, double* s_d) {
+    for (int e = 0; e < n_experts; ++e) {
+        for (int m = 0; m < 2; ++m) {
+            for (int i = 0; i < I; ++i) {
+                int64_t base = (((int64_t)e * 3 + m) * I + i) * H;
+                double amax = 0.0;
+                for (int h = 0; h < H; ++h) {
+                    double v = fabs(load_elem(w, dtype, base + h));
+                    if (v > amax) amax = v;
+                }
+                double sc = pow2_scale(amax);
+                s_gu[((int64_t)e * 2 + m) * I + i] = sc;
+                for (int h = 0; h < H; ++h) q[base + h] = e4m3_encode(load_elem(w, dtype, base + h) / sc);
+            }
+        }
+        int64_t dbase = ((int64_t)e * 3 + 2) * I * (int64_t)H;
+        for (int h = 0; h < H; ++h) {
+            double amax = 0.0;
+            for (int i = 0; i < I; ++i) {
+                double v = fabs(load_elem(w, dtype, dbase + (int64_t)i * H + h));
+                if (v > amax) amax = v;
+            }
+            double sc = pow2_scale(amax);
+            s_d[(int64_t)e * H + h] = sc;
+            for (int i = 0; i < I; ++i)
+                q[dbase + (int64_t)i * H + h] =
+                    e4m3_encode(load_elem(w, dtype, dbase + (int64_t)i * H + h) / sc);
+        }
+    }
+}
+
+/* One expert's FFN on quantized codes (see above).  xq: [H] codes of the
+ * token, sx its scale; q/s_gu/s_d as produced above for expert e. */
+static void expert_ffn_fp8(int H, int I, const uint8_t* xq, double sx, const uint8_t* q,
+                           const double* s_gu, const double* s_d, int e, double clip,
+                           double s_h, double* y) {
+    double* hq = (double*)malloc(sizeof(double) * (size_t)I);
+    for (int i = 0; i < I; ++i) {
+        const uint8_t* gr = q + (((int64_t)e * 3 + 0) * I + i) * H;
+        const uint8_t* ur = q + (((int64_t)e * 3 + 1) * I + i) * H;
+        double g = 0.0, u = 0.0;
+        for (int h = 0; h < H; ++h) {
+            double xv = e4m3_decode(xq[h]);
+            g += xv * e4m3_decode(gr[h]);
+            u += xv * e4m3_decode(ur[h]);
+        }
+        g *= sx * s_gu[((int64_t)e * 2 + 0) * I + i];
+        u *= sx * s_gu[((int64_t)e * 2 + 1) * I + i];
+        g = clamp_keep_nan(g, clip);
+        u = clamp_keep_nan(u, clip);
+        double hv = g / (1.0 + exp(-g)) * u;
+        hq[i] = e4m3_decode(e4m3_encode(hv / s_h));
+    }
+    const uint8_t* dm = q + ((int64_t)e * 3 + 2) * I * (int64_t)H;
+    for (int c = 0; c < H; ++c) y[c] = 0.0;
+    for (int i = 0; i < I; ++i)
+        for (int c = 0; c < H; ++c) y[c] += hq[i] * e4m3_decode(dm[(int64_t)i * H + c]);
+    for (int c = 0; c < H; ++c) y[c] *= s_h * s_d[(int64_t)e * H + c];
+    free(hq);
+}
+
+/*
+ * oracle_forward_fp8: the layer with FP8 expert weights (shared expert too),
+ * routing as in oracle_forward (bf16/fp32 gate, unquantized).  clip > 0 is
+ * required (it bounds h).  q/s_gu/s_d: routed experts; sq/ss_gu/ss_d: the
+ * shared expert (NULL when absent).  out: [n_tok,H]; idx_out/w_out as above.
+ */
+void oracle_forward_fp8(int64_t T, int H, int E, int k, int I, int dtype, const void* x,
+                        const void* gate_w, const float* bias, const uint8_t* q,
+                        const double* s_gu, const double* s_d, const uint8_t* sq,
+                        const double* ss_gu, const double* ss_d, double scale, double clip,
+                        const int64_t* tokens, int64_t n_tok, const int32_t* forced_idx,
+                        double* out, int32_t* idx_out, double* w_out) {
+    (void)T;
+    const double s_h = pow2_scale(clip / (1.0 + exp(-clip)) * clip);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t n = 0; n < n_tok; ++n) {
+        int64_t t = tokens[n];
+        double* l = (double*)malloc(sizeof(double) * (size_t)E);
+        double* p = (double*)malloc(sizeof(double) * (size_t)E);
+        double* y = (double*)malloc(sizeof(double) * (size_t)H);
+        uint8_t* xq = (uint8_t*)malloc((size_t)H);
+        int32_t* idx = (int32_t*)malloc(sizeof(int32_t) * (size_t)k);
+        double* w = (double*)malloc(sizeof(double) * (size_t)k);
+        route_one(t, H, E, k, dtype, x, gate_w, bias, scale, l, p, idx, w);
+        if (forced_idx) {
+            double sum = 0.0;
+            for (int j = 0; j < k; ++j) {
+                idx[j] = forced_idx[n * k + j];
+                sum += p[idx[j]];
+            }
+            for (int j = 0; j < k; ++j) w[j] = scale * p[idx[j]] / sum;
+        }
+        double amax = 0.0;
+        for (int h = 0; h < H; ++h) {
+            double v = fabs(load_elem(x, dtype, t * (int64_t)H + h));
+            if (v > amax) amax = v;
+        }
+        const double sx = pow2_scale(amax);
+        for (int h = 0; h < H; ++h) xq[h] = e4m3_encode(load_elem(x, dtype, t * (int64_t)H + h) / sx);
+        double* o = out + n * (int64_t)H;
+        for (int h = 0; h < H; ++h) o[h] = 0.0;
+        for (int j = 0; j < k; ++j) {
+            expert_ffn_fp8(H, I, xq, sx, q, s_gu, s_d, idx[j], clip, s_h, y);
+            for (int h = 0; h < H; ++h) o[h] += w[j] * y[h];
+        }
+        if (sq) {
+            expert_ffn_fp8(H, I, xq, sx, sq, ss_gu, ss_d, 0, clip, s_h, y);
+            for (int h = 0; h < H; ++h) o[h] += y[h];
+        }
+        if (idx_out) memcpy(idx_out + n * k, idx, sizeof(int32_t) * (size_t)k);
+        if (w_out) memcpy(w_out + n * k, w, sizeof(double) * (size_t)k);
+        free(l);
+        free(p);
+        free(y);
+        free(xq);
+        free(idx);
+        free(w);
+    }
+}
+
 /* Number of OpenMP threads the oracle will use (for reporting). */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

@@ -383,3 +383,89 @@ def test_router_stats_match_torch_composition_and_ema_closed_form():
         ema, tot = s2["ema_counts"], s2["ema_total"]
     np.testing.assert_allclose(ema, m ** 5 * c0 + (1 - m ** 5) * counts, rtol=1e-12)
     assert tot == pytest.approx(m ** 5 * 3.0 + (1 - m ** 5) * cfg.T, rel=1e-13)
+
+
+# ---------------------------------------------------------------- FP8 expert weight pins
+
+def _torch_e4m3(v64: torch.Tensor) -> torch.Tensor:
+    """Round to E4M3 with torch's float8 conversion (a library routine)."""
+    return v64.float().to(torch.float8_e4m3fn).to(torch.float64)
+
+
+def test_e4m3_decode_matches_torch_for_all_codes():
+    codes = torch.arange(256, dtype=torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([oracle.e4m3_decode(c) for c in range(256)])
+    nan = np.isnan(ref)
+    assert (np.isnan(got) == nan).all() and nan.sum() == 2  # 0x7F, 0xFF
+    np.testing.assert_array_equal(got[~nan], ref[~nan])
+    assert oracle.e4m3_decode(0x7E) == 448.0 and oracle.e4m3_decode(0x01) == 2.0 ** -9
+
+
+def test_e4m3_encode_matches_torch_rounding():
+    g = torch.Generator().manual_seed(5)
+    v = torch.cat([torch.randn(4000, generator=g) * s for s in (1e-3, 0.05, 1.0, 30.0, 200.0)])
+    # exact midpoints between neighbouring codes: ties go to the even code
+    mids = torch.tensor([(oracle.e4m3_decode(c) + oracle.e4m3_decode(c + 1)) / 2
+                         for c in range(0, 126)], dtype=torch.float64)
+    v = torch.cat([v.double(), mids, -mids])
+    v = v[v.abs() <= 448.0]  # torch maps out-of-range values to NaN (no saturation)
+    got = torch.tensor([oracle.e4m3_decode(oracle.e4m3_encode(float(a))) for a in v],
+                       dtype=torch.float64)
+    np.testing.assert_array_equal(got.numpy(), _torch_e4m3(v).numpy())
+    # saturation: beyond the largest finite value
+    assert oracle.e4m3_encode(1000.0) == 0x7E and oracle.e4m3_encode(-449.0) == 0xFE
+
+
+def test_pow2_scale_closed_form():
+    assert oracle.pow2_scale(0.0) == 1.0
+    assert oracle.pow2_scale(448.0) == 1.0
+    assert oracle.pow2_scale(448.0 * 1.0001) == 2.0
+    assert oracle.pow2_scale(1.0) == 2.0 ** -8  # 1/448 -> 2^ceil(-8.8) = 2^-8
+    for a in (1e-6, 0.37, 5.0, 1e4):
+        s = oracle.pow2_scale(a)
+        assert a / s <= 448.0 and a / s > 224.0 and math.log2(s) == round(math.log2(s))
+
+
+def test_fp8_forward_matches_torch_composition():
+    """The FP8 layer against the same steps written with torch float8 rounding
+    and float64 matmuls (per-channel power-of-two scales, fixed h scale)."""
+    cfg = small_cfg(T=12, H=128, E=4, k=2, I=64, dtype=torch.bfloat16)
+    inp = make_inputs(cfg, seed=41)
+    q, s_gu, s_d = oracle.quantize_weights_fp8(inp["expert_w"])
+    sq, ss_gu, ss_d = oracle.quantize_weights_fp8(inp["shared_w"].unsqueeze(0))
+    got = oracle.forward_fp8(inp["x"], inp["gate_w"], q, s_gu, s_d, sq[0], ss_gu[0], ss_d[0],
+                             cfg.top_k, cfg.routed_scale, cfg.clip_limit)
+    L = cfg.clip_limit
+
+    def p2(a):
+        return 2.0 ** math.ceil(math.log2(a / 448.0)) if a > 0 else 1.0
+
+    def q_w(w3):  # [3,I,H] float64 -> dequantized gate, up (row scales), down (col scales)
+        g = torch.stack([r / p2(float(r.abs().max())) for r in w3[0]])
+        gs = torch.tensor([p2(float(r.abs().max())) for r in w3[0]], dtype=torch.float64)
+        u = torch.stack([r / p2(float(r.abs().max())) for r in w3[1]])
+        us = torch.tensor([p2(float(r.abs().max())) for r in w3[1]], dtype=torch.float64)
+        ds = torch.tensor([p2(float(c.abs().max())) for c in w3[2].T], dtype=torch.float64)
+        d = w3[2] / ds
+        return _torch_e4m3(g), gs, _torch_e4m3(u), us, _torch_e4m3(d), ds
+
+    s_h = p2(L / (1 + math.exp(-L)) * L)
+
+    def ffn(xq, sx, w3):
+        g, gs, u, us, d, ds = q_w(w3)
+        gg = torch.clamp((xq @ g.T) * sx * gs, -L, L)
+        uu = torch.clamp((xq @ u.T) * sx * us, -L, L)
+        hq = _torch_e4m3(F.silu(gg) * uu / s_h)
+        return (hq @ d) * s_h * ds
+
+    x64 = f64(inp["x"])
+    r = oracle.route(inp["x"], inp["gate_w"], cfg.top_k, cfg.routed_scale)
+    assert (got["idx"] == r["idx"]).all()
+    for t in range(cfg.T):
+        sx = p2(float(x64[t].abs().max()))
+        xq = _torch_e4m3(x64[t:t + 1] / sx)
+        ref = ffn(xq, sx, f64(inp["shared_w"]))[0]
+        for j in range(cfg.top_k):
+            ref = ref + r["w"][t, j] * ffn(xq, sx, f64(inp["expert_w"][r["idx"][t, j]]))[0]
+        np.testing.assert_allclose(got["out"][t], ref.numpy(), rtol=1e-9, atol=1e-12)
