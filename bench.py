@@ -51,28 +51,35 @@ def read_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def layer_counts(cfg, idx_cpu):
-    """Algorithmic FLOPs and bytes of one layer forward, from the actual routing."""
+def layer_counts(cfg, idx_cpu, fp8=False):
+    """Algorithmic FLOPs and bytes of one layer forward, from the actual routing
+    (FP8: one byte per expert weight plus its fp32 channel scales)."""
     T, H, E, I, k, S = cfg.T, cfg.H, cfg.E, cfg.I, cfg.top_k, cfg.num_shared
     b = 2 if cfg.dtype == torch.bfloat16 else 4
     touched = int((torch.bincount(idx_cpu.reshape(-1).long(), minlength=E) > 0).sum())
     flops = T * (2 * H * E + (k + S) * 6 * H * I)
-    bytes_ = (touched + S) * 3 * I * H * b + E * H * b + 2 * T * H * b
+    wbytes = (touched + S) * ((3 * I * H) + (2 * I + H) * 4) if fp8 else \
+        (touched + S) * 3 * I * H * b
+    bytes_ = wbytes + E * H * b + 2 * T * H * b
     return flops, bytes_, touched
 
 
-def gate_up_counts(cfg, touched):
+def gate_up_counts(cfg, touched, fp8=False):
     """Algorithmic FLOPs / bytes of one launch of the grouped gate/up GEMM:
     gate+up weights of every touched expert (+ shared), the permuted token rows
-    and x (shared expert) read once, h written once."""
+    and x (shared expert) read once, h written once (FP8: one byte per
+    element, plus channel and token scales)."""
     T, H, I, k, S = cfg.T, cfg.H, cfg.I, cfg.top_k, cfg.num_shared
     rows = T * (k + S)
     flops = 2 * 2 * rows * H * I
-    bytes_ = (touched + S) * 2 * I * H * 2 + rows * H * 2 + rows * I * 2
+    e = 1 if fp8 else 2
+    bytes_ = (touched + S) * 2 * I * H * e + rows * H * e + rows * I * e
+    if fp8:
+        bytes_ += (touched + S) * 2 * I * 4 + T * 4
     return flops, bytes_
 
 
-def down_counts(cfg, touched, scatter_add=False):
+def down_counts(cfg, touched, scatter_add=False, fp8=False):
     """One launch of the grouped down GEMM: down weights of every touched expert
     (+ shared) and h read once; then either the weighted bf16 rows written once
     (store epilogue) or the fp32 token accumulator read and written once
@@ -80,8 +87,11 @@ def down_counts(cfg, touched, scatter_add=False):
     T, H, I, k, S = cfg.T, cfg.H, cfg.I, cfg.top_k, cfg.num_shared
     rows = T * (k + S)
     flops = 2 * rows * H * I
+    e = 1 if fp8 else 2
     out_bytes = 2 * T * H * 4 if scatter_add else rows * H * 2
-    bytes_ = (touched + S) * I * H * 2 + rows * I * 2 + out_bytes
+    bytes_ = (touched + S) * I * H * e + rows * I * e + out_bytes
+    if fp8:
+        bytes_ += (touched + S) * H * 4
     return flops, bytes_
 
 
@@ -289,14 +299,21 @@ def main():
     ap.add_argument("--config", default="hy4_prefill", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--e2e-steps", type=int, default=None,
+                    help="steps of the end-to-end measurement (default: --steps, so that "
+                         "both run equally long under the power cap)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T of the workload (smaller cases for profiling)")
     ap.add_argument("--experts", type=int, default=None,
                     help="override E of the workload (smaller cases for profiling)")
+    ap.add_argument("--weights", default="bf16", choices=["bf16", "fp8"],
+                    help="expert weights as stored (fp8: E4M3 codes + power-of-two "
+                         "channel scales, moe_forward_fp8)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.e2e_steps is None:
+        args.e2e_steps = args.steps
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -307,7 +324,16 @@ def main():
         cfg = replace(cfg, T=args.tokens or cfg.T, E=args.experts or cfg.E,
                       name=f"{cfg.name}_T{args.tokens or cfg.T}_E{args.experts or cfg.E}")
 
+    fp8 = args.weights == "fp8"
+    if fp8:
+        if cfg.dtype != torch.bfloat16:
+            ap.error("--weights fp8 needs a bf16 workload")
+        from dataclasses import replace
+        cfg = replace(cfg, name=f"{cfg.name}_fp8")
+
     if args.impl == "reference":
+        if fp8:
+            ap.error("the reference arm times the fp64 oracle of the bf16 layer")
         return run_reference(args, cfg, rank, world)
 
     from sparse_moe_layer_06_b200 import moe
@@ -328,15 +354,37 @@ def main():
         from sparse_moe_layer_06_b200.workloads import skew_logit_bias
         inp["logit_bias"] = skew_logit_bias(cfg.E).to(dev)
     p = moe.MoEProblem.from_config(cfg)
-    ws = moe.alloc_workspace(p, moe.MOE_CALL_FORWARD, device=dev)
+    ws = moe.alloc_workspace(p, moe.MOE_CALL_FORWARD_FP8 if fp8 else moe.MOE_CALL_FORWARD,
+                             device=dev)
     out = torch.empty(cfg.T, cfg.H, dtype=cfg.dtype, device=dev)
     idx = torch.empty(cfg.T, cfg.top_k, dtype=torch.int32, device=dev)
     w = torch.empty(cfg.T, cfg.top_k, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
+    if fp8:
+        # weights encoded once, outside the timed region (a load-time step)
+        def quantize(wt):
+            q = torch.empty(wt.shape, dtype=torch.uint8, device=dev)
+            sg = torch.empty(wt.shape[0], 2, cfg.I, dtype=torch.float32, device=dev)
+            sd = torch.empty(wt.shape[0], cfg.H, dtype=torch.float32, device=dev)
+            moe.moe_quantize_weights_fp8(p, wt, q, sg, sd, stream)
+            return q, sg, sd
+        wq = quantize(inp["expert_w"])
+        sq = quantize(inp["shared_w"].unsqueeze(0)) if inp["shared_w"] is not None else \
+            (None, None, None)
+        torch.cuda.synchronize(dev)
+        del inp["expert_w"]
+        torch.cuda.empty_cache()
+
+    def forward(x_in, out_t, s):
+        if fp8:
+            moe.moe_forward_fp8(p, x_in, inp["gate_w"], inp["logit_bias"], *wq, *sq, out_t, idx,
+                                w, ws, s)
+        else:
+            moe.moe_forward(p, x_in, inp["gate_w"], inp["logit_bias"], inp["expert_w"],
+                            inp["shared_w"], out_t, idx, w, ws, s)
 
     def step():
-        moe.moe_forward(p, inp["x"], inp["gate_w"], inp["logit_bias"], inp["expert_w"],
-                        inp["shared_w"], out, idx, w, ws, stream)
+        forward(inp["x"], out, stream)
 
     gpu_index = local if torch.cuda.device_count() > 1 else 0
     clocks = ClockSampler(gpu_index).start()
@@ -397,8 +445,7 @@ def main():
             s_cmp.wait_event(in_done[b])
             if i >= 2:
                 s_cmp.wait_event(out_done[b])  # out_dev[b] was copied out
-            moe.moe_forward(p, x_dev[b], inp["gate_w"], inp["logit_bias"], inp["expert_w"],
-                            inp["shared_w"], out_dev[b], idx, w, ws, s_cmp)
+            forward(x_dev[b], out_dev[b], s_cmp)
             cmp_done[b].record(s_cmp)
             s_out.wait_event(cmp_done[b])
             with torch.cuda.stream(s_out):
@@ -429,8 +476,10 @@ def main():
     peaks, peak_kind = read_peaks()
     hbm_peak = float(peaks["hbm_gbs"])
     tf_peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    if fp8:
+        tf_peak *= 2.0  # E4M3 dense peak: the bf16 measurement x the nominal 4.5/2.25 ratio
     idx_cpu = idx.cpu()
-    flops, bytes_, touched = layer_counts(cfg, idx_cpu)
+    flops, bytes_, touched = layer_counts(cfg, idx_cpu, fp8)
     t_s = ms_per_step / 1e3
     tokens_per_s = whole_job_rate(cfg.T, world, t_s)
     roof_t = max(flops / (tf_peak * 1e12), bytes_ / (hbm_peak * 1e9))
@@ -444,10 +493,10 @@ def main():
     dom_ms = kernel_times[dominant][1] / max(1, kernel_times[dominant][0])
     if dominant == "expert_down_combine_gemm":
         kf, kb = down_counts(cfg, touched, scatter_add=True)
-    elif dominant == "expert_down_gemm":
-        kf, kb = down_counts(cfg, touched)
+    elif dominant in ("expert_down_gemm", "expert_down_gemm_fp8"):
+        kf, kb = down_counts(cfg, touched, fp8=fp8)
     else:
-        kf, kb = gate_up_counts(cfg, touched)
+        kf, kb = gate_up_counts(cfg, touched, fp8)
     dom_s = dom_ms / 1e3
     t_hbm = kb / (hbm_peak * 1e9)
     t_tc = kf / (tf_peak * 1e12)
@@ -462,9 +511,13 @@ def main():
     roof["algorithmic"] = {"bytes": kb, "flops": kf}
     roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" \
         else "fallback"
+    if fp8 and roof["bound"] == "tensor":
+        roof["peak_source"] += ", x2 for E4M3 (nominal ratio)"
 
     cpu_base = None
-    if not args.no_cpu_baseline and world == 1:
+    # (the FP8 variant reports none: encoding the full weight set with the
+    # CPU oracle alone takes minutes)
+    if not args.no_cpu_baseline and world == 1 and not fp8:
         import oracle
         oracle.build()
         cpu_inp = cpu_inputs(inp)
@@ -483,13 +536,15 @@ def main():
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16" if cfg.dtype == torch.bfloat16 else "f32",
+        "dtype": "e4m3" if fp8 else ("bf16" if cfg.dtype == torch.bfloat16 else "f32"),
         "data": "synthetic (seeded N(0,1) tokens, N(0,0.006) weights; random init)",
         "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E,
                    "top_k": cfg.top_k, "I": cfg.I, "num_shared": cfg.num_shared,
                    "global_batch": world * cfg.T, "parallelism": f"replicas x{world}",
+                   "weights": args.weights,
                    "l2": "inputs larger than L2 (expert weights "
-                         f"{cfg.E * 3 * cfg.I * cfg.H * 2 / 1e9:.1f} GB streamed each step)"},
+                         f"{cfg.E * 3 * cfg.I * cfg.H * (1 if fp8 else 2) / 1e9:.1f} GB "
+                         "streamed each step)"},
         "tflops": flops / t_s / 1e12,
         "layer_roofline": {"frac": layer_frac, "frac_nominal_8tbs_2.25pf": roof_t_nominal / t_s,
                            "roofline_ms": roof_t * 1e3, "flops": flops, "bytes": bytes_,

@@ -70,7 +70,8 @@ typedef enum {
     MOE_CALL_FFN = 3,
     MOE_CALL_COMBINE = 4,
     MOE_CALL_FORWARD = 5,
-    MOE_CALL_ROUTER_STATS = 6
+    MOE_CALL_ROUTER_STATS = 6,
+    MOE_CALL_FORWARD_FP8 = 7
 } moe_call;
 
 typedef struct {
@@ -237,6 +238,43 @@ int32_t moe_router_stats(const moe_problem* problem, const void* x, const void* 
                          const float* logit_bias, float* P_out, float* f_out, float* aux_out,
                          float* ema_counts, float* ema_total, float momentum, void* workspace,
                          size_t ws_bytes, void* stream);
+
+/*
+ * FP8 expert weights (page "1M上下文实战：Hy4 preview如何从容处理百万token级长
+ * 文档", section "最快部署 1M 上下文": the official deployment uses FP8
+ * weights).  The pages give no number format; this library uses OCP E4M3
+ * codes with power-of-two scales s = 2^n, n the smallest integer with
+ * 448 * 2^n >= the channel's largest magnitude, so that every encoding
+ * decision is exact:
+ *   gate/up weights: one scale per output row i of each matrix,
+ *   down weights:    one scale per output column h,
+ *   token rows x_t:  one scale per token (computed inside moe_forward_fp8),
+ *   SwiGLU output h: one fixed scale from the clamp bound silu(L) * L.
+ * The expert GEMMs run on tcgen05 kind::f8f6f4 (E4M3 x E4M3, fp32 sums); the
+ * router stays in bf16.
+ *
+ * moe_quantize_weights_fp8 -- encode [n_experts, 3, I, H] weights (problem
+ * dtype; device) into E4M3 codes q (same shape, uint8, device) with scales
+ * scale_gu [n_experts, 2, I] (gate rows, then up rows) and scale_d
+ * [n_experts, H] (fp32, device).  H and I must be multiples of 128.
+ * Run once per weight set (e.g. at load time); nothing is allocated.
+ */
+int32_t moe_quantize_weights_fp8(const moe_problem* problem, int32_t n_experts, const void* w,
+                                 uint8_t* q, float* scale_gu, float* scale_d, void* stream);
+
+/*
+ * moe_forward_fp8 -- moe_forward with FP8 expert (and shared-expert) weights
+ * from moe_quantize_weights_fp8 (shared_*: n_experts = 1, or NULL without a
+ * shared expert).  x, gate_w, out: bf16.  Requires dtype MOE_BF16, H and I
+ * multiples of 128, and clip_limit > 0 (it bounds h).  The combine is the
+ * fixed-order gather (deterministic).  Workspace: MOE_CALL_FORWARD_FP8.
+ */
+int32_t moe_forward_fp8(const moe_problem* problem, const void* x, const void* gate_w,
+                        const float* logit_bias, const uint8_t* expert_q,
+                        const float* expert_scale_gu, const float* expert_scale_d,
+                        const uint8_t* shared_q, const float* shared_scale_gu,
+                        const float* shared_scale_d, void* out, int32_t* topk_idx_out,
+                        float* topk_w_out, void* workspace, size_t ws_bytes, void* stream);
 
 /* Copy the device error word of `workspace` to *status_out (host), waiting
  * for the stream.  Returns MOE_OK or MOE_ERR_CUDA / MOE_ERR_INVALID_ARG. */

@@ -467,33 +467,35 @@ double pow2_scale(double amax) {
  */
 void oracle_quantize_weights_fp8(int n_experts, int I, int H, int dtype, const void* w,
                                  uint8_t* q, double* s_gu, double* s_d) {
-    for (int e = 0; e < n_experts; ++e) {
-        for (int m = 0; m < 2; ++m) {
-            for (int i = 0; i < I; ++i) {
-                int64_t base = (((int64_t)e * 3 + m) * I + i) * H;
-                double amax = 0.0;
-                for (int h = 0; h < H; ++h) {
-                    double v = fabs(load_elem(w, dtype, base + h));
-                    if (v > amax) amax = v;
-                }
-                double sc = pow2_scale(amax);
-                s_gu[((int64_t)e * 2 + m) * I + i] = sc;
-                for (int h = 0; h < H; ++h) q[base + h] = e4m3_encode(load_elem(w, dtype, base + h) / sc);
-            }
-        }
-        int64_t dbase = ((int64_t)e * 3 + 2) * I * (int64_t)H;
+    /* gate and up rows: row r = (e*2 + m)*I + i */
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < (int64_t)n_experts * 2 * I; ++r) {
+        const int64_t e = r / (2 * (int64_t)I), m = (r / I) % 2, i = r % I;
+        const int64_t base = ((e * 3 + m) * I + i) * H;
+        double amax = 0.0;
         for (int h = 0; h < H; ++h) {
-            double amax = 0.0;
-            for (int i = 0; i < I; ++i) {
-                double v = fabs(load_elem(w, dtype, dbase + (int64_t)i * H + h));
-                if (v > amax) amax = v;
-            }
-            double sc = pow2_scale(amax);
-            s_d[(int64_t)e * H + h] = sc;
-            for (int i = 0; i < I; ++i)
-                q[dbase + (int64_t)i * H + h] =
-                    e4m3_encode(load_elem(w, dtype, dbase + (int64_t)i * H + h) / sc);
+            double v = fabs(load_elem(w, dtype, base + h));
+            if (v > amax) amax = v;
         }
+        const double sc = pow2_scale(amax);
+        s_gu[r] = sc;
+        for (int h = 0; h < H; ++h) q[base + h] = e4m3_encode(load_elem(w, dtype, base + h) / sc);
+    }
+    /* down columns: column c = e*H + h */
+#pragma omp parallel for schedule(static)
+    for (int64_t c = 0; c < (int64_t)n_experts * H; ++c) {
+        const int64_t e = c / H, h = c % H;
+        const int64_t dbase = (e * 3 + 2) * I * (int64_t)H;
+        double amax = 0.0;
+        for (int i = 0; i < I; ++i) {
+            double v = fabs(load_elem(w, dtype, dbase + (int64_t)i * H + h));
+            if (v > amax) amax = v;
+        }
+        const double sc = pow2_scale(amax);
+        s_d[c] = sc;
+        for (int i = 0; i < I; ++i)
+            q[dbase + (int64_t)i * H + h] =
+                e4m3_encode(load_elem(w, dtype, dbase + (int64_t)i * H + h) / sc);
     }
 }
 

@@ -120,6 +120,15 @@ struct GemmArgs {
     // rows gather_tok[b_row + i] instead of from tmB0 (the permuted copy)
     const int32_t* gather_tok;
     const void* gather_src;
+    // FP8 (E4M3) operands: per weight-channel scales (EPI_SWIGLU: gate then up
+    // row scales, 2*M_total per segment; EPI_DOWN_*: column scales, M_total per
+    // segment), the shared expert's scales, per-token scales of the token rows
+    // (EPI_SWIGLU) and the fixed scale of h (EPI_DOWN_*)
+    const float* scale_w;
+    const float* scale_w_special;
+    const float* token_scale;
+    float h_scale;      // a power of two
+    float h_scale_inv;  // its exact reciprocal
     int32_t* status;           // device error word
 };
 
@@ -129,7 +138,9 @@ struct GemmArgs {
 //         EPI_SWIGLU (MB = 2), else 1 or 2 adjacent 128-row blocks of one
 //         matrix (two MMAs sharing each token tile)
 // The pipeline depth is whatever fits the 227 KB of shared memory.
-template <int EPI, int NMAX, int MB>
+//   FP8   E4M3 operands (kind::f8f6f4): 128 K-elements per 128-byte row per
+//         stage instead of 64, scales applied in the epilogue
+template <int EPI, int NMAX, int MB, bool FP8 = false>
 struct GemmCfg {
     static_assert(NMAX % 16 == 0 && NMAX >= 16 && NMAX <= 256, "N tile");
     static_assert(MB == 1 || MB == 2, "weight sub-tiles");
@@ -137,6 +148,7 @@ struct GemmCfg {
     static constexpr bool kSwiGLU = (EPI == EPI_SWIGLU);
     static constexpr bool kDown = (EPI == EPI_DOWN_ATOMIC || EPI == EPI_DOWN_STORE);
     static constexpr int kNumA = MB;
+    static constexpr int kKStep = FP8 ? 128 : 64;  // K elements per stage (128-byte rows)
     static constexpr int kATileBytes = 128 * 128;  // 128 rows x 64 bf16
     static constexpr int kABytes = kNumA * kATileBytes;
     static constexpr int kBBytes = NMAX * 128;  // NMAX rows x 64 bf16
@@ -156,7 +168,8 @@ struct GemmCfg {
     static constexpr int kBarrierBytes = 512;
     // (rounded to 128 bytes so that what follows stays 128-byte aligned)
     static constexpr int kSchedBytes = (5 * (kMaxSegments + 1) * 4 + 127) / 128 * 128;
-    static constexpr int kMetaBytes = kDown ? 2 * NMAX * 8 : 0;
+    static constexpr bool kMeta = kDown || (kSwiGLU && FP8);  // per-column metadata
+    static constexpr int kMetaBytes = kMeta ? 2 * NMAX * 8 : 0;
     static constexpr int kEpiWarps = 8;
     // EPI_SWIGLU: token index of each row of the current tile (row gather)
     static constexpr int kGatherBytes = kSwiGLU ? NMAX * 4 : 0;
@@ -224,9 +237,9 @@ __device__ __forceinline__ float clamp_keep_nan(float v, float lim) {
     return v > lim ? lim : (v < -lim ? -lim : v);
 }
 
-template <int EPI, int NMAX, int MB>
+template <int EPI, int NMAX, int MB, bool FP8>
 __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs args) {
-    using C = GemmCfg<EPI, NMAX, MB>;
+    using C = GemmCfg<EPI, NMAX, MB, FP8>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned ring (the 128-byte swizzle atoms need it)
     uint8_t* ring = reinterpret_cast<uint8_t*>(
@@ -301,7 +314,7 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
     constexpr int kRowsPerTile = C::kSwiGLU ? 128 : 128 * MB;
     const int nblk = (args.M_total + kRowsPerTile - 1) / kRowsPerTile;
     const int total_tiles = ss.prefix[nseg] * nblk;
-    const int ksteps = args.K / 64;
+    const int ksteps = args.K / C::kKStep;
 
     auto fail = [&](int code) {
         *abort_flag = 1;
@@ -329,7 +342,8 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
             const CUtensorMap* tA = ti.special ? &args.tmA1 : &args.tmA0;
             const CUtensorMap* tB = ti.special ? args.tmB1 : args.tmB0;
             const int a_base = ti.special ? 0 : ti.seg * args.a_seg_stride;
-            const bool gather = C::kSwiGLU && args.gather_tok != nullptr && !ti.special;
+            const bool gather =
+                C::kSwiGLU && !FP8 && args.gather_tok != nullptr && !ti.special;
             if (gather) {
                 __syncwarp();  // the previous tile's rows are all issued
                 for (int i = lane; i < ti.n_mma; i += 32)
@@ -348,7 +362,7 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
                 }
                 uint8_t* sA = ring + stage * C::kStageBytes;
                 uint8_t* sB = sA + C::kABytes;
-                const int k0 = kb * 64;
+                const int k0 = kb * C::kKStep;
                 if (gather) {
                     const int chunk = lane & 7;
                     for (int r = lane >> 3; r < ti.n_mma; r += 4) {
@@ -370,10 +384,11 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
                     armed |= 1u << stage;
                     armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
                     if constexpr (C::kDown) {
-                        // MN-major A: one 3D copy of 2*MB chunks of 64 H-values
-                        // x 64 K-rows, chunk-major in shared memory (8 KB each)
+                        // MN-major A: one 3D copy of the tile's 128-byte-wide H
+                        // chunks (bf16: 2*MB chunks of 64 values x 64 K-rows;
+                        // FP8: MB chunks of 128 values x 128 K-rows), chunk-major
                         ptx::tma_load_3d(sA, tA, 0, a_base + args.a_off0 + k0,
-                                         ti.blk * 2 * MB, &full_bar[stage], pol_w);
+                                         ti.blk * (FP8 ? MB : 2 * MB), &full_bar[stage], pol_w);
                     } else if constexpr (C::kSwiGLU) {
                         // gate and up tiles (adjacent matrices) in one 3D copy
                         ptx::tma_load_3d(sA, tA, k0, ti.blk * 128, a_base + args.a_off0,
@@ -420,6 +435,11 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
             uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
             bool ok = true;
             constexpr uint32_t kAMajor = C::kDown ? 1u : 0u;
+            // MN-major A: per MMA (K = 16 bf16 / 32 FP8) the next 16 / 32 K-rows
+            // of 128 bytes; between 128-byte H chunks 8 KB (bf16: two chunks per
+            // 128-row sub-tile) -- unused for FP8, where one chunk is 128 rows
+            constexpr uint32_t kMnStep = FP8 ? 4096u : 2048u;
+            constexpr uint32_t kMnLbo = FP8 ? 16384u : 8192u;
             for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
                 TileInfo ti;
                 if (!decode_tile(t, nblk, nseg, ss, args.special_seg, ti)) continue;
@@ -429,7 +449,8 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
                 }
                 ptx::tc_fence_after();
                 const uint32_t d0 = tmem_base + acc * C::kAccCols;
-                const uint32_t idesc = ptx::idesc_bf16_f32(128, ti.n_mma, kAMajor, 0);
+                const uint32_t idesc = FP8 ? ptx::idesc_e4m3_f32(128, ti.n_mma, kAMajor, 0)
+                                           : ptx::idesc_bf16_f32(128, ti.n_mma, kAMajor, 0);
                 for (int kb = 0; kb < ksteps; ++kb) {
                     if (!ptx::mbar_wait(&full_bar[stage], phase, abort_flag)) {
                         fail(DEV_ERR_TIMEOUT);
@@ -450,9 +471,10 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
                         for (int j = 0; j < MB; ++j) {
                             const uint32_t a_sub = a_addr + j * C::kATileBytes;
                             const uint64_t adesc =
-                                C::kDown ? ptx::smem_desc_sw128(a_sub + kk * 2048, 8192, 1024)
+                                C::kDown ? ptx::smem_desc_sw128(a_sub + kk * kMnStep, kMnLbo, 1024)
                                          : ptx::smem_desc_sw128(a_sub + kk * 32, 16, 1024);
-                            ptx::mma_bf16(d0 + j * NMAX, adesc, bdesc, idesc, accum);
+                            if constexpr (FP8) ptx::mma_fp8(d0 + j * NMAX, adesc, bdesc, idesc, accum);
+                            else ptx::mma_bf16(d0 + j * NMAX, adesc, bdesc, idesc, accum);
                         }
                     }
                     ptx::mma_commit(&empty_bar[stage]);
@@ -484,7 +506,7 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
             if (!decode_tile(t, nblk, nseg, ss, args.special_seg, ti)) continue;
             int32_t* w_tok = reinterpret_cast<int32_t*>(s_meta) + mi * 2 * NMAX;
             float* w_wt = reinterpret_cast<float*>(w_tok + NMAX);
-            if constexpr (C::kDown) {
+            if constexpr (C::kMeta) {
                 // token and routing weight of every column, fetched by the
                 // epilogue warps together before the accumulator is ready, so
                 // the loads overlap the main loop.  Two buffers alternate by
@@ -502,6 +524,7 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
                         tok = r - args.routed_rows;
                         wt = 1.0f;
                     }
+                    if (args.token_scale) wt *= __ldg(args.token_scale + tok);
                     w_tok[c] = tok;
                     w_wt[c] = wt;
                 }
@@ -530,15 +553,34 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
                 const bool odd = lane & 1;
                 const int m_pair = m - (odd ? 1 : 0);
                 __nv_bfloat16* hout = reinterpret_cast<__nv_bfloat16*>(args.out);
+                // FP8: gate and up channel scales of this lane's row
+                float sg = 1.0f, su = 1.0f;
+                if constexpr (FP8) {
+                    const float* sc = ti.special ? args.scale_w_special
+                                                 : args.scale_w + static_cast<size_t>(ti.seg) * 2 *
+                                                                      args.M_total;
+                    if (m_ok) {
+                        sg = __ldg(sc + m);
+                        su = __ldg(sc + args.M_total + m);
+                    }
+                }
                 auto emit = [&](float (&g)[16], float (&u)[16], int c0) {
                     float hv[16];
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
-                        const float gg = clamp_keep_nan(g[j], args.clip);
-                        const float uu = clamp_keep_nan(u[j], args.clip);
+                        float gin = g[j], uin = u[j];
+                        if constexpr (FP8) {
+                            // token scale (per column) x channel scale (per lane)
+                            const float ts = w_wt[c0 + j];
+                            gin *= ts * sg;
+                            uin *= ts * su;
+                        }
+                        const float gg = clamp_keep_nan(gin, args.clip);
+                        const float uu = clamp_keep_nan(uin, args.clip);
                         // silu(g) = g / (1 + e^-g): approximate exp2 and
                         // reciprocal (both ~1e-7 relative, far below bf16)
                         hv[j] = gg * fast_rcp(1.0f + __expf(-gg)) * uu;
+                        if constexpr (FP8) hv[j] *= args.h_scale_inv;  // exact: power of two
                     }
 #pragma unroll
                     for (int j = 0; j < 16; j += 2) {
@@ -548,12 +590,18 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
                         const float send = odd ? hv[j] : hv[j + 1];
                         const float other = __shfl_xor_sync(0xffffffffu, send, 1);
                         const int col = c0 + j + (odd ? 1 : 0);
-                        const __nv_bfloat162 pr = odd ? __floats2bfloat162_rn(other, mine)
-                                                      : __floats2bfloat162_rn(mine, other);
+                        const float lo = odd ? other : mine;
+                        const float hi = odd ? mine : other;
                         if (m_ok && col < ti.n_valid) {
-                            *reinterpret_cast<__nv_bfloat162*>(
-                                hout + static_cast<size_t>(ti.out_row + col) * args.out_ld +
-                                m_pair) = pr;
+                            const size_t o =
+                                static_cast<size_t>(ti.out_row + col) * args.out_ld + m_pair;
+                            if constexpr (FP8) {
+                                *reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(args.out) +
+                                                             o) = ptx::e4m3x2(lo, hi);
+                            } else {
+                                *reinterpret_cast<__nv_bfloat162*>(hout + o) =
+                                    __floats2bfloat162_rn(lo, hi);
+                            }
                         }
                     }
                 };
@@ -593,6 +641,14 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
                 for (int sub = 0; sub < MB; ++sub) {
                     const int m = (ti.blk * MB + sub) * 128 + row_in_tile;
                     const bool m_ok = m < args.M_total;
+                    // FP8: h scale x this lane's weight-column scale
+                    float lane_scale = 1.0f;
+                    if constexpr (FP8 && C::kDown) {
+                        const float* sc = ti.special ? args.scale_w_special
+                                                     : args.scale_w + static_cast<size_t>(ti.seg) *
+                                                                          args.M_total;
+                        if (m_ok) lane_scale = args.h_scale * __ldg(sc + m);
+                    }
                     for (int c0 = half * 16; c0 < ti.n_mma; c0 += 32) {
                         float v[16];
                         ptx::tmem_ld16(tbase + sub * NMAX + c0, v);
@@ -623,8 +679,8 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
 #pragma unroll
                             for (int j = 0; j < 16; j += 2) {
                                 const int c = c0 + j;
-                                const float a0 = v[j] * w_wt[c];
-                                const float a1 = v[j + 1] * w_wt[c + 1];
+                                const float a0 = v[j] * lane_scale * w_wt[c];
+                                const float a1 = v[j + 1] * lane_scale * w_wt[c + 1];
                                 const float mine = odd ? a1 : a0;
                                 const float send = odd ? a0 : a1;
                                 const float other = __shfl_xor_sync(0xffffffffu, send, 1);

@@ -101,32 +101,45 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2D bf16 row-major [rows, cols] tensor, box = 64 columns x box_rows rows,
-// 128-byte swizzle, zero fill outside the tensor.
-bool make_tmap(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int box_rows) {
+// Element type of a tensor map: bf16 (2 bytes) or FP8 codes (1 byte).  A
+// 128-byte swizzled row holds 128 / bytes elements.
+struct ElemType {
+    CUtensorMapDataType dt;
+    int bytes;
+};
+constexpr ElemType kBF16{CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2};
+constexpr ElemType kU8{CU_TENSOR_MAP_DATA_TYPE_UINT8, 1};
+
+// 2D row-major [rows, cols] tensor, box = one 128-byte row segment x box_rows
+// rows, 128-byte swizzle, zero fill outside the tensor.
+bool make_tmap(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int box_rows,
+               ElemType et = kBF16) {
     EncodeTiledFn fn = encode_fn();
     if (!fn || rows <= 0 || cols <= 0) return false;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
-    cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * et.bytes};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / et.bytes),
+                         static_cast<cuuint32_t>(box_rows)};
     cuuint32_t estr[2] = {1u, 1u};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    CUresult r = fn(m, et.dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
 // Gate/up weights as a 3D bf16 tensor {H, I, n_mats} (n_mats [I,H] matrices
 // back to back), box {64, 128, 2}: one copy brings the gate and the up tile.
-bool make_tmap_gateup(CUtensorMap* m, const void* ptr, int64_t n_mats, int64_t I, int64_t H) {
+bool make_tmap_gateup(CUtensorMap* m, const void* ptr, int64_t n_mats, int64_t I, int64_t H,
+                      ElemType et = kBF16) {
     EncodeTiledFn fn = encode_fn();
     if (!fn || n_mats <= 0) return false;
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(I),
                           static_cast<cuuint64_t>(n_mats)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(H) * 2, static_cast<cuuint64_t>(I * H) * 2};
-    cuuint32_t box[3] = {64u, 128u, 2u};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(H) * et.bytes,
+                             static_cast<cuuint64_t>(I * H) * et.bytes};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / et.bytes), 128u, 2u};
     cuuint32_t estr[3] = {1u, 1u, 1u};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+    CUresult r = fn(m, et.dt, 3, const_cast<void*>(ptr), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -136,23 +149,29 @@ bool make_tmap_gateup(CUtensorMap* m, const void* ptr, int64_t n_mats, int64_t I
 // H/64}: dim 0 = 64 consecutive H values, dim 1 = the row (stride H*2 bytes),
 // dim 2 = which 64-wide H chunk (stride 128 bytes).  A {64, 64, 2*mb} box is
 // one K-step of 2*mb chunks, laid out chunk by chunk in shared memory.
-bool make_tmap_down(CUtensorMap* m, const void* ptr, int64_t rows, int64_t H, int mb) {
+bool make_tmap_down(CUtensorMap* m, const void* ptr, int64_t rows, int64_t H, int mb,
+                    ElemType et = kBF16) {
     EncodeTiledFn fn = encode_fn();
-    if (!fn || rows <= 0 || H % 64 != 0) return false;
-    cuuint64_t dims[3] = {64u, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(H / 64)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(H) * 2, 128u};
-    cuuint32_t box[3] = {64u, 64u, static_cast<cuuint32_t>(2 * mb)};
+    const int64_t chunk = 128 / et.bytes;  // H values per 128-byte chunk
+    if (!fn || rows <= 0 || H % chunk != 0) return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(chunk), static_cast<cuuint64_t>(rows),
+                          static_cast<cuuint64_t>(H / chunk)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(H) * et.bytes, 128u};
+    // one K-step: 64 (bf16) or 128 (FP8) rows of each of the tile's chunks
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(chunk), static_cast<cuuint32_t>(chunk),
+                         static_cast<cuuint32_t>(et.bytes == 2 ? 2 * mb : mb)};
     cuuint32_t estr[3] = {1u, 1u, 1u};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+    CUresult r = fn(m, et.dt, 3, const_cast<void*>(ptr), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
 // The token-row operand with the five box heights 16 << j.
-bool make_tmap_rows(CUtensorMap* maps, const void* ptr, int64_t rows, int64_t cols) {
+bool make_tmap_rows(CUtensorMap* maps, const void* ptr, int64_t rows, int64_t cols,
+                    ElemType et = kBF16) {
     for (int j = 0; j < kNumBoxSizes; ++j)
-        if (!make_tmap(&maps[j], ptr, rows, cols, 16 << j)) return false;
+        if (!make_tmap(&maps[j], ptr, rows, cols, 16 << j, et)) return false;
     return true;
 }
 
@@ -258,7 +277,7 @@ struct Carve {
 
 struct Layout {
     size_t status, logits, idx, w, hist, base, counts, offsets, partial, sched_gu, sched_dn, pos, src, row_w;
-    size_t x_perm, x_bf16, w_bf16, ws_bf16, h_perm, out_acc, y_perm, total;
+    size_t x_perm, x_bf16, w_bf16, ws_bf16, h_perm, out_acc, y_perm, x_q, s_x, total;
 };
 
 int64_t perm_chunks(int64_t T) { return (T + kPermTokens - 1) / kPermTokens; }
@@ -299,6 +318,25 @@ Layout layout_for(const moe_problem* p, int call, int64_t ffn_rows = 0, int ffn_
             L.partial = c.take(((T + kStatsTokensPerBlock - 1) / kStatsTokensPerBlock) * E * 4);
             L.counts = c.take(E * 4);
             break;
+        case MOE_CALL_FORWARD_FP8:
+            L.logits = c.take(T * E * 4);
+            L.idx = c.take(T * k * 4);
+            L.w = c.take(T * k * 4);
+            L.hist = c.take(perm_chunks(T) * E * 4);
+            L.base = c.take(perm_chunks(T) * E * 4);
+            L.counts = c.take(E * 4);
+            L.offsets = c.take((E + 1) * 4);
+            L.sched_gu = c.take(sched_bytes());
+            L.sched_dn = c.take(sched_bytes());
+            L.pos = c.take(T * k * 4);
+            L.src = c.take(T * k * 4);
+            L.row_w = c.take(T * k * 4);
+            L.x_q = c.take(T * H);
+            L.s_x = c.take(T * 4);
+            L.x_perm = c.take(T * k * H);
+            L.h_perm = c.take(T * (k + S) * I);
+            L.y_perm = c.take(T * (k + S) * H * 2);
+            break;
         case MOE_CALL_FORWARD:
         default:
             L.logits = c.take(T * E * 4);
@@ -337,35 +375,49 @@ T* at(void* ws, size_t off) {
 
 // ------------------------------------------------------------------ GEMM launch
 
-template <int EPI, int NMAX, int MB>
+template <int EPI, int NMAX, int MB, bool FP8 = false>
 int32_t launch_gemm_n(const GemmArgs& a, int grid, cudaStream_t s, const char* name) {
-    using C = GemmCfg<EPI, NMAX, MB>;
+    using C = GemmCfg<EPI, NMAX, MB, FP8>;
     int dev = 0;
     cudaGetDevice(&dev);
     static std::atomic<uint64_t> configured{0};
     const uint64_t bit = (dev < 64) ? (1ull << dev) : 0;
     if (!bit || !(configured.load() & bit)) {
-        if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI, NMAX, MB>,
+        if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI, NMAX, MB, FP8>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::kSmemBytes) != cudaSuccess)
             return MOE_ERR_CUDA;
         configured.fetch_or(bit);
     }
     MOE_LAUNCH(name, s,
-               grouped_gemm_kernel<EPI, NMAX, MB><<<grid, C::kThreads, C::kSmemBytes, s>>>(a));
+               grouped_gemm_kernel<EPI, NMAX, MB, FP8><<<grid, C::kThreads, C::kSmemBytes, s>>>(a));
     return MOE_OK;
 }
 
-template <int EPI, int MB>
+template <int EPI, int MB, bool FP8 = false>
 int32_t launch_gemm_mb(int nmax, const GemmArgs& a, int grid, cudaStream_t s, const char* name) {
     switch (nmax) {
-        case 16: return launch_gemm_n<EPI, 16, MB>(a, grid, s, name);
-        case 32: return launch_gemm_n<EPI, 32, MB>(a, grid, s, name);
-        case 64: return launch_gemm_n<EPI, 64, MB>(a, grid, s, name);
-        case 128: return launch_gemm_n<EPI, 128, MB>(a, grid, s, name);
-        case 160: return launch_gemm_n<EPI, 160, MB>(a, grid, s, name);
-        case 256: return launch_gemm_n<EPI, 256, MB>(a, grid, s, name);
+        case 16: return launch_gemm_n<EPI, 16, MB, FP8>(a, grid, s, name);
+        case 32: return launch_gemm_n<EPI, 32, MB, FP8>(a, grid, s, name);
+        case 64: return launch_gemm_n<EPI, 64, MB, FP8>(a, grid, s, name);
+        case 128: return launch_gemm_n<EPI, 128, MB, FP8>(a, grid, s, name);
+        case 160: return launch_gemm_n<EPI, 160, MB, FP8>(a, grid, s, name);
+        case 256: return launch_gemm_n<EPI, 256, MB, FP8>(a, grid, s, name);
         default: return MOE_ERR_UNSUPPORTED;
+    }
+}
+
+// FP8 expert GEMMs: gate/up (+SwiGLU) and down with the store epilogue.
+template <int EPI>
+int32_t launch_gemm_fp8(int nmax, int mb, const GemmArgs& a, int64_t max_tiles, cudaStream_t s,
+                        const char* name) {
+    int grid = static_cast<int>(std::min<int64_t>(sm_count(), std::max<int64_t>(1, max_tiles)));
+    if constexpr (EPI == EPI_SWIGLU) {
+        return launch_gemm_mb<EPI, 2, true>(nmax, a, grid, s, name);
+    } else {
+        static_assert(EPI == EPI_DOWN_STORE, "FP8 down GEMM uses the store epilogue");
+        if (mb == 2) return launch_gemm_mb<EPI, 2, true>(nmax, a, grid, s, name);
+        return launch_gemm_mb<EPI, 1, true>(nmax, a, grid, s, name);
     }
 }
 
@@ -639,7 +691,7 @@ const char* moe_status_string(int32_t status) {
 
 size_t moe_workspace_size(const moe_problem* p, int32_t call) {
     if (check_problem(p) != MOE_OK) return 0;
-    if (call < MOE_CALL_ROUTE || call > MOE_CALL_ROUTER_STATS) return 0;
+    if (call < MOE_CALL_ROUTE || call > MOE_CALL_FORWARD_FP8) return 0;
     if (call == MOE_CALL_FFN) {
         // the FFN workspace depends on rows/groups; size it for the routed
         // rows of this problem (T*top_k) and E groups, the larger of the two
@@ -1059,6 +1111,177 @@ int32_t moe_router_stats(const moe_problem* p, const void* x, const void* gate_w
                router_stats_final_kernel<<<1, kMaxExperts, 0, s>>>(
                    partial, nblocks, counts, p->T, p->E, p->top_k, momentum, P_out, f_out,
                    aux_out, ema_counts, ema_total));
+    return MOE_OK;
+}
+
+int32_t moe_quantize_weights_fp8(const moe_problem* p, int32_t n_experts, const void* w,
+                                 uint8_t* q, float* scale_gu, float* scale_d, void* stream) {
+    MOE_TRY(check_problem(p));
+    if (!w || !q || !scale_gu || !scale_d) return MOE_ERR_INVALID_ARG;
+    if (n_experts < 1) return MOE_ERR_INVALID_ARG;
+    if (p->H % 128 != 0 || p->I % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t I = p->I, H = p->H, n = n_experts;
+    // gate and up rows: groups of 2*I rows out of every 3*I
+    const int64_t rows = n * 2 * I;
+    const unsigned rblocks = static_cast<unsigned>((rows + 7) / 8);
+    // down columns: one thread per (expert, column)
+    const unsigned cblocks = static_cast<unsigned>((n * H + 255) / 256);
+    if (p->dtype == MOE_BF16) {
+        const __nv_bfloat16* wb = static_cast<const __nv_bfloat16*>(w);
+        MOE_LAUNCH("quantize_weight_rows", s,
+                   quantize_rows_e4m3_kernel<__nv_bfloat16><<<rblocks, 256, 0, s>>>(
+                       wb, rows, static_cast<int>(H), 2 * I, 3 * I, q, scale_gu));
+        MOE_LAUNCH("quantize_weight_cols", s,
+                   quantize_cols_e4m3_kernel<__nv_bfloat16><<<cblocks, 256, 0, s>>>(
+                       wb + 2 * I * H, 3 * I * H, 3 * I * H, static_cast<int>(n),
+                       static_cast<int>(I), static_cast<int>(H), q + 2 * I * H, scale_d));
+    } else {
+        const float* wf = static_cast<const float*>(w);
+        MOE_LAUNCH("quantize_weight_rows", s,
+                   quantize_rows_e4m3_kernel<float><<<rblocks, 256, 0, s>>>(
+                       wf, rows, static_cast<int>(H), 2 * I, 3 * I, q, scale_gu));
+        MOE_LAUNCH("quantize_weight_cols", s,
+                   quantize_cols_e4m3_kernel<float><<<cblocks, 256, 0, s>>>(
+                       wf + 2 * I * H, 3 * I * H, 3 * I * H, static_cast<int>(n),
+                       static_cast<int>(I), static_cast<int>(H), q + 2 * I * H, scale_d));
+    }
+    return MOE_OK;
+}
+
+int32_t moe_forward_fp8(const moe_problem* p, const void* x, const void* gate_w,
+                        const float* bias, const uint8_t* expert_q, const float* expert_s_gu,
+                        const float* expert_s_d, const uint8_t* shared_q,
+                        const float* shared_s_gu, const float* shared_s_d, void* out,
+                        int32_t* idx_out, float* w_out, void* ws, size_t ws_bytes,
+                        void* stream) {
+    MOE_TRY(check_problem(p));
+    if (p->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (p->H % 128 != 0 || p->I % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    if (!(p->clip_limit > 0.0f && std::isfinite(p->clip_limit))) return MOE_ERR_UNSUPPORTED;
+    if (!x || !gate_w || !expert_q || !expert_s_gu || !expert_s_d || !out || !ws)
+        return MOE_ERR_INVALID_ARG;
+    if (p->num_shared && (!shared_q || !shared_s_gu || !shared_s_d)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(gate_w) || !aligned16(expert_q) || !aligned16(out) ||
+        !aligned16(ws) || (shared_q && !aligned16(shared_q)))
+        return MOE_ERR_INVALID_ARG;
+    const Layout L = layout_for(p, MOE_CALL_FORWARD_FP8);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    if (p->T == 0) return MOE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t* status = at<int32_t>(ws, L.status);
+    const int64_t T = p->T, H = p->H, E = p->E, I = p->I, k = p->top_k, S = p->num_shared;
+    int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, L.idx);
+    float* w = w_out ? w_out : at<float>(ws, L.w);
+
+    // 1. route (bf16 gate GEMM, unquantized)
+    MOE_TRY(run_logits(p, x, gate_w, at<float>(ws, L.logits), status, s));
+    MOE_TRY(run_topk(p, at<float>(ws, L.logits), bias, idx, w, s));
+    // 2. dispatch
+    const int nmax = pick_nmax(static_cast<double>(T * k) / E);
+    const int nmax_dn = pick_down_nmax(nmax);
+    int32_t* sg = at<int32_t>(ws, L.sched_gu);
+    int32_t* sd = at<int32_t>(ws, L.sched_dn);
+    int32_t* pos = at<int32_t>(ws, L.pos);
+    int32_t* src = at<int32_t>(ws, L.src);
+    float* row_w = at<float>(ws, L.row_w);
+    MOE_TRY(run_dispatch(p, idx, w, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base),
+                         at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets), sg, nmax, sd,
+                         nmax_dn, pos, src, row_w, status, s));
+    // 3. token rows to E4M3 with a power-of-two scale per token, then permuted
+    uint8_t* x_q = at<uint8_t>(ws, L.x_q);
+    float* s_x = at<float>(ws, L.s_x);
+    MOE_LAUNCH("quantize_tokens", s,
+               quantize_rows_e4m3_kernel<__nv_bfloat16><<<static_cast<unsigned>((T + 7) / 8), 256,
+                                                          0, s>>>(
+                   static_cast<const __nv_bfloat16*>(x), T, static_cast<int>(H), T, T, x_q, s_x));
+    uint8_t* x_perm = at<uint8_t>(ws, L.x_perm);
+    MOE_TRY((run_gather<uint8_t, uint8_t>(x_q, T, p->H, p->top_k, pos, T * k, x_perm, nullptr,
+                                          nullptr, s)));
+    // 4. gate/up on E4M3 codes; the epilogue applies token x channel scales,
+    //    clamps, and writes h as E4M3 with the fixed power-of-two scale
+    const double L_clip = p->clip_limit;
+    const double hmax = L_clip / (1.0 + std::exp(-L_clip)) * L_clip;
+    const float h_scale = static_cast<float>(std::ldexp(1.0, static_cast<int>(
+                                                                 std::ceil(std::log2(hmax / 448.0)))));
+    uint8_t* h = at<uint8_t>(ws, L.h_perm);
+    const int64_t h_rows = T * (k + S);
+    const int nseg = static_cast<int>(E + S);
+    {
+        GemmArgs a = base_args(status);
+        if (!make_tmap_gateup(&a.tmA0, expert_q, E * 3, I, H, kU8)) return MOE_ERR_CUDA;
+        if (!make_tmap_rows(a.tmB0, x_perm, T * k, H, kU8)) return MOE_ERR_CUDA;
+        if (S) {
+            if (!make_tmap_gateup(&a.tmA1, shared_q, 3, I, H, kU8)) return MOE_ERR_CUDA;
+            if (!make_tmap_rows(a.tmB1, x_q, T, H, kU8)) return MOE_ERR_CUDA;
+        } else {
+            a.tmA1 = a.tmA0;
+            for (int j = 0; j < kNumBoxSizes; ++j) a.tmB1[j] = a.tmB0[j];
+        }
+        a.sched = sg;
+        a.nseg = nseg;
+        a.special_seg = S ? static_cast<int32_t>(E) : -1;
+        a.K = static_cast<int32_t>(H);
+        a.M_total = static_cast<int32_t>(I);
+        a.a_seg_stride = 3;
+        a.a_off0 = 0;
+        a.out = h;
+        a.out_ld = static_cast<int32_t>(I);
+        a.clip = effective_clip(p);
+        a.row_token = src;
+        a.routed_rows = static_cast<int32_t>(T * k);
+        a.token_scale = s_x;
+        a.scale_w = expert_s_gu;
+        a.scale_w_special = shared_s_gu;
+        a.h_scale = h_scale;
+        a.h_scale_inv = 1.0f / h_scale;
+        MOE_TRY(launch_gemm_fp8<EPI_SWIGLU>(nmax, 2, a, max_tiles(h_rows, nseg, nmax, I), s,
+                                            "expert_gate_up_gemm_fp8"));
+    }
+    // 5. down on E4M3 codes; epilogue: h scale x column scale x routing weight
+    __nv_bfloat16* y_perm = at<__nv_bfloat16>(ws, L.y_perm);
+    {
+        GemmArgs a = base_args(status);
+        const int mb = pick_down_mb(nmax_dn);
+        if (!make_tmap_down(&a.tmA0, expert_q, E * 3 * I, H, mb, kU8)) return MOE_ERR_CUDA;
+        if (!make_tmap_rows(a.tmB0, h, h_rows, I, kU8)) return MOE_ERR_CUDA;
+        if (S) {
+            if (!make_tmap_down(&a.tmA1, shared_q, 3 * I, H, mb, kU8)) return MOE_ERR_CUDA;
+        } else {
+            a.tmA1 = a.tmA0;
+        }
+        for (int j = 0; j < kNumBoxSizes; ++j) a.tmB1[j] = a.tmB0[j];
+        a.sched = sd;
+        a.nseg = nseg;
+        a.special_seg = S ? static_cast<int32_t>(E) : -1;
+        a.K = static_cast<int32_t>(I);
+        a.M_total = static_cast<int32_t>(H);
+        a.a_seg_stride = static_cast<int32_t>(3 * I);
+        a.a_off0 = static_cast<int32_t>(2 * I);
+        a.out = y_perm;
+        a.out_ld = static_cast<int32_t>(H);
+        a.n_tokens = static_cast<int32_t>(T);
+        a.row_token = src;
+        a.row_weight = row_w;
+        a.routed_rows = static_cast<int32_t>(T * k);
+        a.scale_w = expert_s_d;
+        a.scale_w_special = shared_s_d;
+        a.h_scale = h_scale;
+        a.h_scale_inv = 1.0f / h_scale;
+        MOE_TRY(launch_gemm_fp8<EPI_DOWN_STORE>(nmax_dn, mb, a,
+                                                max_tiles(h_rows, nseg, nmax_dn, H, 128 * mb), s,
+                                                "expert_down_gemm_fp8"));
+    }
+    // 6. fixed-order combine into token order
+    {
+        const int warps = 8;
+        const int64_t segs = (H / 8 + kSegVecs - 1) / kSegVecs;
+        const unsigned blocks = static_cast<unsigned>((T * segs + warps - 1) / warps);
+        MOE_LAUNCH("combine_gather", s,
+                   gather_sum_kernel<__nv_bfloat16><<<blocks, warps * 32, 0, s>>>(
+                       y_perm, pos, T, p->H, p->top_k, T * k, S ? T * k : -1,
+                       static_cast<__nv_bfloat16*>(out), status));
+    }
     return MOE_OK;
 }
 

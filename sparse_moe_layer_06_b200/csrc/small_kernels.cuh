@@ -559,6 +559,83 @@ __global__ void gather_sum_kernel(const __nv_bfloat16* __restrict__ y,
     }
 }
 
+// ------------------------------------------------------------------ FP8 (E4M3) quantization
+//
+// Scales are powers of two, s = 2^n with n the smallest integer such that
+// 448 * 2^n >= amax (448 is the largest E4M3 value; s = 1 when amax == 0), so
+// v / s is exact and the E4M3 code of v / s does not depend on the precision
+// the division is done in.
+
+__device__ __forceinline__ float pow2_scale_f(float amax) {
+    if (!(amax > 0.0f)) return 1.0f;
+    int n = ilogbf(amax) - 8;  // 2^8 < 448 < 2^9
+    while (ldexpf(448.0f, n) < amax) ++n;
+    while (n > -126 && ldexpf(448.0f, n - 1) >= amax) --n;
+    return ldexpf(1.0f, n);
+}
+
+template <typename T>
+__device__ __forceinline__ float load_f32(const T* p, int64_t i);
+template <>
+__device__ __forceinline__ float load_f32<float>(const float* p, int64_t i) {
+    return p[i];
+}
+template <>
+__device__ __forceinline__ float load_f32<__nv_bfloat16>(const __nv_bfloat16* p, int64_t i) {
+    return __bfloat162float(p[i]);
+}
+
+// Per-row quantization: for each of n_rows rows of length len (one warp per
+// row), scale = pow2_scale(max |row|), codes = e4m3(row / scale).
+// Row r of the output is row (r / group) * src_group_stride + r % group of the
+// input (group = src_group_stride: plain rows; group = 2*I, stride 3*I: the
+// gate and up rows of [E,3,I,H] expert weights); codes keep the input's layout.
+template <typename T>
+__global__ void quantize_rows_e4m3_kernel(const T* __restrict__ in, int64_t n_rows, int len,
+                                          int64_t group, int64_t src_group_stride,
+                                          uint8_t* __restrict__ q, float* __restrict__ scale) {
+    const int lane = threadIdx.x & 31;
+    const int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (r >= n_rows) return;
+    const int64_t src_row = (r / group) * src_group_stride + r % group;
+    const T* row = in + src_row * len;
+    float amax = 0.0f;
+    for (int i = lane; i < len; i += 32) amax = fmaxf(amax, fabsf(load_f32(row, i)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float sc = pow2_scale_f(amax);
+    const float inv = 1.0f / sc;  // exact: power of two
+    uint8_t* qr = q + src_row * len;
+    for (int i = 2 * lane; i < len; i += 64) {
+        const uint16_t two = ptx::e4m3x2(load_f32(row, i) * inv, load_f32(row, i + 1) * inv);
+        *reinterpret_cast<uint16_t*>(qr + i) = two;
+    }
+    if (lane == 0) scale[r] = sc;
+}
+
+// Per-column quantization of [n_mats][rows][cols] matrices: each thread owns
+// one column of one matrix: scale = pow2_scale(max |column|).
+template <typename T>
+__global__ void quantize_cols_e4m3_kernel(const T* __restrict__ in, int64_t mat_stride,
+                                          int64_t out_mat_stride, int n_mats, int rows, int cols,
+                                          uint8_t* __restrict__ q, float* __restrict__ scale) {
+    const int64_t id = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (id >= static_cast<int64_t>(n_mats) * cols) return;
+    const int mat = static_cast<int>(id / cols);
+    const int c = static_cast<int>(id - static_cast<int64_t>(mat) * cols);
+    const T* base = in + mat * mat_stride + c;
+    float amax = 0.0f;
+    for (int r = 0; r < rows; ++r) amax = fmaxf(amax, fabsf(load_f32(base, static_cast<int64_t>(r) * cols)));
+    const float sc = pow2_scale_f(amax);
+    const float inv = 1.0f / sc;
+    uint8_t* qb = q + mat * out_mat_stride + c;
+    for (int r = 0; r < rows; ++r)
+        qb[static_cast<int64_t>(r) * cols] =
+            static_cast<uint8_t>(ptx::e4m3x2(load_f32(base, static_cast<int64_t>(r) * cols) * inv,
+                                             0.0f) & 0xFF);
+    scale[id] = sc;
+}
+
 __global__ void cast_f32_bf16_kernel(const float* __restrict__ in, __nv_bfloat16* __restrict__ out,
                                      int64_t n) {
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;

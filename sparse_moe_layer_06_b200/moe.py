@@ -25,13 +25,13 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE = 0, 1, 2, 3
 MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_BAD_INDEX = 4, 5, 6
 MOE_F32, MOE_BF16 = 0, 1
 (MOE_CALL_ROUTE, MOE_CALL_ROUTER_LOGITS, MOE_CALL_PERMUTE, MOE_CALL_FFN, MOE_CALL_COMBINE,
- MOE_CALL_FORWARD, MOE_CALL_ROUTER_STATS) = range(7)
+ MOE_CALL_FORWARD, MOE_CALL_ROUTER_STATS, MOE_CALL_FORWARD_FP8) = range(8)
 
 EXPORTED = (
     "moe_workspace_size", "moe_status_string", "moe_router_logits", "moe_route", "moe_permute",
     "moe_grouped_swiglu_ffn", "moe_combine", "moe_forward", "moe_read_device_status",
     "moe_clear_device_status", "moe_launch_count", "moe_profile_start", "moe_profile_stop",
-    "moe_route_noalloc", "moe_router_stats",
+    "moe_route_noalloc", "moe_router_stats", "moe_quantize_weights_fp8", "moe_forward_fp8",
 )
 ROUTE_NOALLOC_SCRATCH_BYTES = 1 << 20
 
@@ -113,6 +113,8 @@ def load_library(path: str = LIB_PATH):
             "moe_profile_stop": (I32, [ctypes.POINTER(KernelTimeC), I32, ctypes.POINTER(I32)]),
             "moe_route_noalloc": (I32, [PP, P, P, P, P, P, P]),
             "moe_router_stats": (I32, [PP, P, P, P, P, P, P, P, P, ctypes.c_float, P, SZ, P]),
+            "moe_quantize_weights_fp8": (I32, [PP, I32, P, P, P, P, P]),
+            "moe_forward_fp8": (I32, [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -209,6 +211,34 @@ def moe_router_stats(problem, x, gate_w, logit_bias, P_out, f_out, aux_out, ema_
         _ptr(ema_total, torch.float32, "ema_total", optional=True), float(momentum),
         _ptr(workspace, None, "workspace"), workspace.numel(), _stream(stream)),
         "moe_router_stats")
+
+
+def moe_quantize_weights_fp8(problem, w, q, scale_gu, scale_d, stream=None):
+    """Encode [n,3,I,H] weights into E4M3 codes q (uint8, same shape) with
+    scale_gu [n,2,I] and scale_d [n,H] (fp32); n is w.shape[0]."""
+    pc = problem.c()
+    _check(load_library().moe_quantize_weights_fp8(
+        ctypes.byref(pc), int(w.shape[0]), _ptr(w, problem.dtype, "w"),
+        _ptr(q, torch.uint8, "q"), _ptr(scale_gu, torch.float32, "scale_gu"),
+        _ptr(scale_d, torch.float32, "scale_d"), _stream(stream)), "moe_quantize_weights_fp8")
+
+
+def moe_forward_fp8(problem, x, gate_w, logit_bias, expert_q, expert_s_gu, expert_s_d,
+                    shared_q, shared_s_gu, shared_s_d, out, topk_idx_out, topk_w_out, workspace,
+                    stream=None):
+    pc = problem.c()
+    _check(load_library().moe_forward_fp8(
+        ctypes.byref(pc), _ptr(x, torch.bfloat16, "x"), _ptr(gate_w, torch.bfloat16, "gate_w"),
+        _ptr(logit_bias, torch.float32, "logit_bias", optional=True),
+        _ptr(expert_q, torch.uint8, "expert_q"), _ptr(expert_s_gu, torch.float32, "expert_s_gu"),
+        _ptr(expert_s_d, torch.float32, "expert_s_d"),
+        _ptr(shared_q, torch.uint8, "shared_q", optional=True),
+        _ptr(shared_s_gu, torch.float32, "shared_s_gu", optional=True),
+        _ptr(shared_s_d, torch.float32, "shared_s_d", optional=True),
+        _ptr(out, torch.bfloat16, "out"),
+        _ptr(topk_idx_out, torch.int32, "topk_idx_out", optional=True),
+        _ptr(topk_w_out, torch.float32, "topk_w_out", optional=True),
+        _ptr(workspace, None, "workspace"), workspace.numel(), _stream(stream)), "moe_forward_fp8")
 
 
 def moe_permute(problem, topk_idx, x, offsets, pos, src_token, x_perm, workspace, stream=None):
