@@ -332,6 +332,9 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
             args.l2_hints ? ptx::policy_evict_first() : ptx::policy_evict_normal();
         const uint64_t pol_x =
             args.l2_hints ? ptx::policy_evict_last() : ptx::policy_evict_normal();
+        // the special (shared-expert) segment's weights are re-read by every
+        // token chunk of that segment: keep them in L2 rather than streaming
+        const uint64_t pol_ws = pol_x;
         const bf16_raw_ptr gsrc = reinterpret_cast<bf16_raw_ptr>(args.gather_src);
         uint32_t stage = 0, phase = 0;
         uint32_t armed = 0, armed_phase = 0;  // per-stage bits (lane 0)
@@ -342,6 +345,7 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
             const CUtensorMap* tA = ti.special ? &args.tmA1 : &args.tmA0;
             const CUtensorMap* tB = ti.special ? args.tmB1 : args.tmB0;
             const int a_base = ti.special ? 0 : ti.seg * args.a_seg_stride;
+            const uint64_t pw = ti.special ? pol_ws : pol_w;
             const bool gather =
                 C::kSwiGLU && !FP8 && args.gather_tok != nullptr && !ti.special;
             if (gather) {
@@ -388,18 +392,18 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
                         // chunks (bf16: 2*MB chunks of 64 values x 64 K-rows;
                         // FP8: MB chunks of 128 values x 128 K-rows), chunk-major
                         ptx::tma_load_3d(sA, tA, 0, a_base + args.a_off0 + k0,
-                                         ti.blk * (FP8 ? MB : 2 * MB), &full_bar[stage], pol_w);
+                                         ti.blk * (FP8 ? MB : 2 * MB), &full_bar[stage], pw);
                     } else if constexpr (C::kSwiGLU) {
                         // gate and up tiles (adjacent matrices) in one 3D copy
                         ptx::tma_load_3d(sA, tA, k0, ti.blk * 128, a_base + args.a_off0,
-                                         &full_bar[stage], pol_w);
+                                         &full_bar[stage], pw);
                     } else if constexpr (MB == 2) {
                         // both 128-row blocks in one 256-row box
                         ptx::tma_load_2d(sA, tA, k0, a_base + args.a_off0 + ti.blk * 256,
-                                         &full_bar[stage], pol_w);
+                                         &full_bar[stage], pw);
                     } else {
                         ptx::tma_load_2d(sA, tA, k0, a_base + args.a_off0 + ti.blk * 128,
-                                         &full_bar[stage], pol_w);
+                                         &full_bar[stage], pw);
                     }
                     if (!gather) {
                         int q = 0;
