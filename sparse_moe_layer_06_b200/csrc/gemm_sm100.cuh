@@ -115,6 +115,10 @@ struct GemmArgs {
     float clip;                // EPI_SWIGLU clamp limit (+inf: none)
     int32_t out_f32;           // EPI_DOWN_STORE: fp32 (1) or bf16 (0) output
     int32_t l2_hints;          // 1: weights evict-first, token rows evict-last; 0: none
+    // EPI_LOGITS: the K range split into k_splits parts (>= 1, <= K / 64), one
+    // tile each; part s writes its partial sums at out + s * split_stride
+    int32_t k_splits;
+    int64_t split_stride;
     // EPI_SWIGLU row gather: when gather_tok != nullptr, ordinary segments
     // take their token rows straight from gather_src ([n_tokens, K] bf16) at
     // rows gather_tok[b_row + i] instead of from tmB0 (the permuted copy)
@@ -313,7 +317,9 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
     // matrices at the same rows, other sub-tiles are adjacent row blocks
     constexpr int kRowsPerTile = C::kSwiGLU ? 128 : 128 * MB;
     const int nblk = (args.M_total + kRowsPerTile - 1) / kRowsPerTile;
-    const int total_tiles = ss.prefix[nseg] * nblk;
+    // EPI_LOGITS may split K: tile t covers K part t % ksplit of tile t / ksplit
+    const int ksplit = (EPI == EPI_LOGITS && args.k_splits > 1) ? args.k_splits : 1;
+    const int total_tiles = ss.prefix[nseg] * nblk * ksplit;
     const int ksteps = args.K / C::kKStep;
 
     auto fail = [&](int code) {
@@ -341,7 +347,9 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
         bool ok = true;
         for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
             TileInfo ti;
-            if (!decode_tile(t, nblk, nseg, ss, args.special_seg, ti)) continue;
+            const int ks = t % ksplit;
+            if (!decode_tile(t / ksplit, nblk, nseg, ss, args.special_seg, ti)) continue;
+            const int kb_begin = ks * ksteps / ksplit, kb_end = (ks + 1) * ksteps / ksplit;
             const CUtensorMap* tA = ti.special ? &args.tmA1 : &args.tmA0;
             const CUtensorMap* tB = ti.special ? args.tmB1 : args.tmB0;
             const int a_base = ti.special ? 0 : ti.seg * args.a_seg_stride;
@@ -355,7 +363,7 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
                 __syncwarp();
             }
             const uint32_t bytes = C::kABytes + (gather ? 0 : ti.n_mma * 128);
-            for (int kb = 0; kb < ksteps; ++kb) {
+            for (int kb = kb_begin; kb < kb_end; ++kb) {
                 int got = 1;
                 if (lane == 0) got = ptx::mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag);
                 got = __shfl_sync(0xffffffffu, got, 0);
@@ -446,7 +454,9 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
             constexpr uint32_t kMnLbo = FP8 ? 16384u : 8192u;
             for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
                 TileInfo ti;
-                if (!decode_tile(t, nblk, nseg, ss, args.special_seg, ti)) continue;
+                const int ks = t % ksplit;
+                if (!decode_tile(t / ksplit, nblk, nseg, ss, args.special_seg, ti)) continue;
+                const int kb_begin = ks * ksteps / ksplit, kb_end = (ks + 1) * ksteps / ksplit;
                 if (!ptx::mbar_wait(&acce_bar[acc], acc_phase ^ 1, abort_flag)) {
                     fail(DEV_ERR_TIMEOUT);
                     break;
@@ -455,7 +465,7 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
                 const uint32_t d0 = tmem_base + acc * C::kAccCols;
                 const uint32_t idesc = FP8 ? ptx::idesc_e4m3_f32(128, ti.n_mma, kAMajor, 0)
                                            : ptx::idesc_bf16_f32(128, ti.n_mma, kAMajor, 0);
-                for (int kb = 0; kb < ksteps; ++kb) {
+                for (int kb = kb_begin; kb < kb_end; ++kb) {
                     if (!ptx::mbar_wait(&full_bar[stage], phase, abort_flag)) {
                         fail(DEV_ERR_TIMEOUT);
                         ok = false;
@@ -469,7 +479,7 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
                     const uint32_t b_addr = a_addr + C::kABytes;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
-                        const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+                        const uint32_t accum = (kb > kb_begin || kk > 0) ? 1u : 0u;
                         const uint64_t bdesc = ptx::smem_desc_sw128(b_addr + kk * 32, 16, 1024);
 #pragma unroll
                         for (int j = 0; j < MB; ++j) {
@@ -507,7 +517,8 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
         uint32_t mi = 0, meta_phase = 0;
         for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
             TileInfo ti;
-            if (!decode_tile(t, nblk, nseg, ss, args.special_seg, ti)) continue;
+            const int ks = t % ksplit;
+            if (!decode_tile(t / ksplit, nblk, nseg, ss, args.special_seg, ti)) continue;
             int32_t* w_tok = reinterpret_cast<int32_t*>(s_meta) + mi * 2 * NMAX;
             float* w_wt = reinterpret_cast<float*>(w_tok + NMAX);
             if constexpr (C::kMeta) {
@@ -704,7 +715,8 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
                                     const size_t o =
                                         static_cast<size_t>(ti.out_row + c0 + j) * args.out_ld + m;
                                     if constexpr (EPI == EPI_LOGITS) {
-                                        reinterpret_cast<float*>(args.out)[o] = v[j];
+                                        reinterpret_cast<float*>(args.out)[o + ks * args.split_stride] =
+                                            v[j];
                                     } else {
                                         reinterpret_cast<float*>(args.out)[o] = v[j] * w_wt[c0 + j];
                                     }

@@ -255,14 +255,32 @@ int pick_down_mb(int nmax) {
     return 2;
 }
 
-// Router logits: 256 experts per tile (both 128-row blocks in one 256-row
-// box) against 32 tokens, so a 4096-token batch spreads over 128 CTAs.
-// MOE_LOGITS_NMAX=64 selects 64-token tiles.
-int logits_nmax() {
-    static const int v = env_int("MOE_LOGITS_NMAX", 32) == 64 ? 64 : 32;
-    return v;
+// Router logits GEMM shape: the gate weight (E rows, one or two 128-row
+// sub-tiles) against token chunks of 256 (32/64 for small batches).  With the
+// problem's own workspace the K range is also split so that about one tile per
+// SM runs (at most 8 parts): every CTA then reads only its part of the gate
+// weight and of the chunk, instead of the whole 3 MB weight per 32 tokens.
+// The parts land in separate fp32 slices that the top-k kernel sums in a fixed
+// order.  The split depends only on the problem, so the workspace size does too.
+constexpr int64_t kSplitTargetTiles = 148;  // SMs of a B200
+struct LogitsPlan {
+    int nmax, mb, splits;
+};
+LogitsPlan logits_plan(const moe_problem* p, bool allow_split) {
+    LogitsPlan lp;
+    lp.mb = p->E > 128 ? 2 : 1;
+    lp.nmax = p->T >= 256 ? 256 : (p->T > 32 ? 64 : 32);
+    lp.splits = 1;
+    if (allow_split && p->dtype == MOE_BF16) {
+        const int64_t chunks = (p->T + lp.nmax - 1) / lp.nmax;
+        const int64_t nblk = (p->E + 128 * lp.mb - 1) / (128 * lp.mb);
+        const int64_t base = std::max<int64_t>(1, chunks * nblk);
+        const int64_t sp = std::min<int64_t>(kSplitTargetTiles / base, std::min<int64_t>(8, p->H / 64));
+        lp.splits = static_cast<int>(std::max<int64_t>(1, sp));
+    }
+    return lp;
 }
-constexpr int kLogitsMb = 2;
+
 
 // ------------------------------------------------------------------ workspace layout
 
@@ -293,7 +311,7 @@ Layout layout_for(const moe_problem* p, int call, int64_t ffn_rows = 0, int ffn_
         case MOE_CALL_ROUTER_LOGITS:
             break;
         case MOE_CALL_ROUTE:
-            L.logits = c.take(T * E * 4);
+            L.logits = c.take(logits_plan(p, true).splits * T * E * 4);
             break;
         case MOE_CALL_PERMUTE:
             L.hist = c.take(perm_chunks(T) * E * 4);
@@ -312,14 +330,14 @@ Layout layout_for(const moe_problem* p, int call, int64_t ffn_rows = 0, int ffn_
         case MOE_CALL_COMBINE:
             break;
         case MOE_CALL_ROUTER_STATS:
-            L.logits = c.take(T * E * 4);
+            L.logits = c.take(logits_plan(p, true).splits * T * E * 4);
             L.idx = c.take(T * k * 4);
             L.w = c.take(T * k * 4);
             L.partial = c.take(((T + kStatsTokensPerBlock - 1) / kStatsTokensPerBlock) * E * 4);
             L.counts = c.take(E * 4);
             break;
         case MOE_CALL_FORWARD_FP8:
-            L.logits = c.take(T * E * 4);
+            L.logits = c.take(logits_plan(p, true).splits * T * E * 4);
             L.idx = c.take(T * k * 4);
             L.w = c.take(T * k * 4);
             L.hist = c.take(perm_chunks(T) * E * 4);
@@ -339,7 +357,7 @@ Layout layout_for(const moe_problem* p, int call, int64_t ffn_rows = 0, int ffn_
             break;
         case MOE_CALL_FORWARD:
         default:
-            L.logits = c.take(T * E * 4);
+            L.logits = c.take(logits_plan(p, true).splits * T * E * 4);
             L.idx = c.take(T * k * 4);
             L.w = c.take(T * k * 4);
             L.hist = c.take(perm_chunks(T) * E * 4);
@@ -429,6 +447,10 @@ int32_t launch_gemm(int nmax, int mb, const GemmArgs& a, int64_t max_tiles, cuda
     if constexpr (EPI == EPI_SWIGLU) {
         return launch_gemm_mb<EPI, 2>(nmax, a, grid, s, name);
     } else if constexpr (EPI == EPI_LOGITS) {
+        if (nmax == 256) {
+            if (mb == 2) return launch_gemm_n<EPI, 256, 2>(a, grid, s, name);
+            return launch_gemm_n<EPI, 256, 1>(a, grid, s, name);
+        }
         if (nmax == 64) {
             if (mb == 2) return launch_gemm_n<EPI, 64, 2>(a, grid, s, name);
             return launch_gemm_n<EPI, 64, 1>(a, grid, s, name);
@@ -490,29 +512,34 @@ GemmArgs base_args(int32_t* status) {
 
 // Router logits through tcgen05 (bf16 x and gate weight).
 int32_t run_logits_bf16(const moe_problem* p, const void* x, const void* gate_w, float* logits,
-                        int32_t* status, cudaStream_t s) {
+                        int32_t* status, cudaStream_t s, const LogitsPlan& lp) {
     GemmArgs a = base_args(status);
-    const int mb = (p->E > 128) ? kLogitsMb : 1;
-    if (!make_tmap(&a.tmA0, gate_w, p->E, p->H, 128 * mb)) return MOE_ERR_CUDA;
+    if (!make_tmap(&a.tmA0, gate_w, p->E, p->H, 128 * lp.mb)) return MOE_ERR_CUDA;
     if (!make_tmap_rows(a.tmB0, x, p->T, p->H)) return MOE_ERR_CUDA;
     a.tmA1 = a.tmA0;
     for (int j = 0; j < kNumBoxSizes; ++j) a.tmB1[j] = a.tmB0[j];
     a.sched = nullptr;
     a.single_rows = static_cast<int32_t>(p->T);
-    const int lnmax = logits_nmax();
-    a.single_chunk_len = lnmax;
+    a.single_chunk_len = lp.nmax;
     a.nseg = 1;
     a.K = p->H;
     a.M_total = p->E;
     a.out = logits;
     a.out_ld = p->E;
-    return launch_gemm<EPI_LOGITS>(lnmax, mb, a, max_tiles(p->T, 1, lnmax, p->E, 128 * mb), s,
-                                   "router_logits_gemm");
+    a.k_splits = lp.splits;
+    a.split_stride = p->T * static_cast<int64_t>(p->E);
+    return launch_gemm<EPI_LOGITS>(
+        lp.nmax, lp.mb, a, max_tiles(p->T, 1, lp.nmax, p->E, 128 * lp.mb) * lp.splits, s,
+        "router_logits_gemm");
 }
 
+// Router logits into `logits`; with split = true (the problem's own workspace)
+// the K parts go to consecutive [T,E] slices (logits_plan(p, true).splits of
+// them) for run_topk to sum.
 int32_t run_logits(const moe_problem* p, const void* x, const void* gate_w, float* logits,
-                   int32_t* status, cudaStream_t s) {
-    if (p->dtype == MOE_BF16) return run_logits_bf16(p, x, gate_w, logits, status, s);
+                   int32_t* status, cudaStream_t s, bool split = false) {
+    if (p->dtype == MOE_BF16)
+        return run_logits_bf16(p, x, gate_w, logits, status, s, logits_plan(p, split));
     MOE_LAUNCH("router_logits_f32", s,
                router_logits_f32_kernel<<<static_cast<unsigned>(p->T), 256, 0, s>>>(
                    static_cast<const float*>(x), static_cast<const float*>(gate_w), p->H, p->E,
@@ -520,13 +547,16 @@ int32_t run_logits(const moe_problem* p, const void* x, const void* gate_w, floa
     return MOE_OK;
 }
 
-int32_t run_topk(const moe_problem* p, const float* logits, const float* bias, int32_t* idx,
-                 float* w, cudaStream_t s) {
+// Top-k over the logits; n_parts > 1 sums that many [T,E] slices first (in
+// slice order) and leaves the sum in the first slice.
+int32_t run_topk(const moe_problem* p, float* logits, const float* bias, int32_t* idx, float* w,
+                 cudaStream_t s, int n_parts = 1) {
     const int warps = 8;
     const unsigned blocks = static_cast<unsigned>((p->T + warps - 1) / warps);
     MOE_LAUNCH("route_topk", s,
-               topk_kernel<<<blocks, warps * 32, 0, s>>>(logits, bias, p->T, p->E, p->top_k,
-                                                         p->routed_scale, idx, w));
+               topk_kernel<<<blocks, warps * 32, 0, s>>>(logits, n_parts, p->T * p->E, bias, p->T,
+                                                         p->E, p->top_k, p->routed_scale, idx,
+                                                         w));
     return MOE_OK;
 }
 
@@ -725,8 +755,8 @@ int32_t moe_route(const moe_problem* p, const void* x, const void* gate_w, const
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int32_t* status = at<int32_t>(ws, L.status);
     float* logits = at<float>(ws, L.logits);
-    MOE_TRY(run_logits(p, x, gate_w, logits, status, s));
-    return run_topk(p, logits, bias, topk_idx, topk_w, s);
+    MOE_TRY(run_logits(p, x, gate_w, logits, status, s, true));
+    return run_topk(p, logits, bias, topk_idx, topk_w, s, logits_plan(p, true).splits);
 }
 
 int32_t moe_permute(const moe_problem* p, const int32_t* topk_idx, const void* x,
@@ -899,8 +929,8 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
     }
 
     // 1. route
-    MOE_TRY(run_logits(p, x, gate_w, logits, status, s));
-    MOE_TRY(run_topk(p, logits, bias, idx, w, s));
+    MOE_TRY(run_logits(p, x, gate_w, logits, status, s, true));
+    MOE_TRY(run_topk(p, logits, bias, idx, w, s, logits_plan(p, true).splits));
 
     // 2. dispatch bookkeeping + schedules
     const int nmax = pick_nmax(static_cast<double>(T * k) / E);
@@ -1100,8 +1130,9 @@ int32_t moe_router_stats(const moe_problem* p, const void* x, const void* gate_w
     int32_t* idx = at<int32_t>(ws, L.idx);
     int32_t* counts = at<int32_t>(ws, L.counts);
     float* partial = at<float>(ws, L.partial);
-    MOE_TRY(run_logits(p, x, gate_w, logits, status, s));
-    MOE_TRY(run_topk(p, logits, bias, idx, at<float>(ws, L.w), s));
+    MOE_TRY(run_logits(p, x, gate_w, logits, status, s, true));
+    MOE_TRY(run_topk(p, logits, bias, idx, at<float>(ws, L.w), s,
+                     logits_plan(p, true).splits));
     if (cudaMemsetAsync(counts, 0, p->E * sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
     const int nblocks = static_cast<int>((p->T + kStatsTokensPerBlock - 1) / kStatsTokensPerBlock);
     MOE_LAUNCH("router_prob_partial", s,
@@ -1175,8 +1206,9 @@ int32_t moe_forward_fp8(const moe_problem* p, const void* x, const void* gate_w,
     float* w = w_out ? w_out : at<float>(ws, L.w);
 
     // 1. route (bf16 gate GEMM, unquantized)
-    MOE_TRY(run_logits(p, x, gate_w, at<float>(ws, L.logits), status, s));
-    MOE_TRY(run_topk(p, at<float>(ws, L.logits), bias, idx, w, s));
+    MOE_TRY(run_logits(p, x, gate_w, at<float>(ws, L.logits), status, s, true));
+    MOE_TRY(run_topk(p, at<float>(ws, L.logits), bias, idx, w, s,
+                     logits_plan(p, true).splits));
     // 2. dispatch
     const int nmax = pick_nmax(static_cast<double>(T * k) / E);
     const int nmax_dn = pick_down_nmax(nmax);
