@@ -144,7 +144,7 @@ struct GemmArgs {
 // The pipeline depth is whatever fits the 227 KB of shared memory.
 //   FP8   E4M3 operands (kind::f8f6f4): 128 K-elements per 128-byte row per
 //         stage instead of 64, scales applied in the epilogue
-template <int EPI, int NMAX, int MB, bool FP8 = false>
+template <int EPI, int NMAX, int MB, bool FP8 = false, bool PAIR = false>
 struct GemmCfg {
     static_assert(NMAX % 16 == 0 && NMAX >= 16 && NMAX <= 256, "N tile");
     static_assert(MB == 1 || MB == 2, "weight sub-tiles");
@@ -155,7 +155,12 @@ struct GemmCfg {
     static constexpr int kKStep = FP8 ? 128 : 64;  // K elements per stage (128-byte rows)
     static constexpr int kATileBytes = 128 * 128;  // 128 rows x 64 bf16
     static constexpr int kABytes = kNumA * kATileBytes;
-    static constexpr int kBBytes = NMAX * 128;  // NMAX rows x 64 bf16
+    // PAIR: the two CTAs of a cluster run one tile with cta_group::2 MMAs of
+    // M = 256 (each CTA its 128 weight rows of every sub-tile) and each CTA
+    // holds half of the NMAX token rows
+    static_assert(!PAIR || (NMAX % 32 == 0 && EPI != EPI_LOGITS), "pair tile");
+    static constexpr int kBRows = PAIR ? NMAX / 2 : NMAX;
+    static constexpr int kBBytes = kBRows * 128;  // token rows x 128 bytes
     static constexpr int kStageBytes = kABytes + kBBytes;
     static_assert(kStageBytes % 1024 == 0, "stage alignment");
     static constexpr int kAccCols = kNumA * NMAX;  // sub-tile j at column j*NMAX
@@ -241,9 +246,10 @@ __device__ __forceinline__ float clamp_keep_nan(float v, float lim) {
     return v > lim ? lim : (v < -lim ? -lim : v);
 }
 
-template <int EPI, int NMAX, int MB, bool FP8>
+template <int EPI, int NMAX, int MB, bool FP8, bool PAIR>
 __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs args) {
-    using C = GemmCfg<EPI, NMAX, MB, FP8>;
+    using C = GemmCfg<EPI, NMAX, MB, FP8, PAIR>;
+    constexpr int CG = PAIR ? 2 : 1;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned ring (the 128-byte swizzle atoms need it)
     uint8_t* ring = reinterpret_cast<uint8_t*>(
@@ -264,6 +270,11 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int nseg = args.sched ? args.nseg : 1;
+    // PAIR: rank 0 of the cluster (the leader) issues the MMAs for both CTAs;
+    // both walk the same tile sequence, one cluster per unit of the grid
+    const uint32_t rank = PAIR ? ptx::cluster_ctarank() : 0u;
+    const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+    const int units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
     SmemSched ss;
     ss.prefix = s_sched;
     ss.b_row0 = s_sched + (nseg + 1);
@@ -289,7 +300,8 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
         }
         for (int a = 0; a < 2; ++a) {
             ptx::mbar_init(&accf_bar[a], 1);
-            ptx::mbar_init(&acce_bar[a], C::kEpiWarps);
+            // PAIR: the leader's MMA waits for the epilogues of both CTAs
+            ptx::mbar_init(&acce_bar[a], PAIR ? 2 * C::kEpiWarps : C::kEpiWarps);
         }
         ptx::mbar_init(final_bar, 1);
         ptx::mbar_init(&metaf_bar[0], C::kEpiWarps);
@@ -305,18 +317,22 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
         ptx::prefetch_tmap(m);
     }
     if (warp == 1) {
-        ptx::tmem_alloc(tmem_slot, C::kTmemCols);
-        ptx::tmem_relinquish();
+        ptx::tmem_alloc<CG>(tmem_slot, C::kTmemCols);
+        ptx::tmem_relinquish<CG>();
     }
     ptx::tc_fence_before();
-    __syncthreads();
+    // PAIR: both CTAs' barriers and TMEM exist before either touches the other's
+    if constexpr (PAIR) ptx::cluster_sync();
+    else __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
     // a tile covers 128 weight rows per sub-tile; gate/up sub-tiles are the two
     // matrices at the same rows, other sub-tiles are adjacent row blocks
     constexpr int kRowsPerTile = C::kSwiGLU ? 128 : 128 * MB;
-    const int nblk = (args.M_total + kRowsPerTile - 1) / kRowsPerTile;
+    const int nblk_cta = (args.M_total + kRowsPerTile - 1) / kRowsPerTile;
+    // PAIR: a tile is a pair of adjacent weight blocks, CTA r taking block 2p + r
+    const int nblk = PAIR ? (nblk_cta + 1) / 2 : nblk_cta;
     // EPI_LOGITS may split K: tile t covers K part t % ksplit of tile t / ksplit
     const int ksplit = (EPI == EPI_LOGITS && args.k_splits > 1) ? args.k_splits : 1;
     const int total_tiles = ss.prefix[nseg] * nblk * ksplit;
@@ -325,6 +341,15 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
     auto fail = [&](int code) {
         *abort_flag = 1;
         set_device_error(args.status, code);
+    };
+    // tile t -> this CTA's share of it (all roles decode the same way)
+    auto decode = [&](int t, TileInfo& ti) -> bool {
+        if (!decode_tile(t / ksplit, nblk, nseg, ss, args.special_seg, ti)) return false;
+        if constexpr (PAIR) {
+            ti.blk = 2 * ti.blk + static_cast<int>(rank);
+            ti.n_mma = (ti.n_valid + 31) & ~31;  // N split in two multiples of 16
+        }
+        return true;
     };
 
     if (warp == 0) {
@@ -345,24 +370,29 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
         uint32_t stage = 0, phase = 0;
         uint32_t armed = 0, armed_phase = 0;  // per-stage bits (lane 0)
         bool ok = true;
-        for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
+        for (int t = unit; ok && t < total_tiles; t += units) {
             TileInfo ti;
             const int ks = t % ksplit;
-            if (!decode_tile(t / ksplit, nblk, nseg, ss, args.special_seg, ti)) continue;
+            if (!decode(t, ti)) continue;
             const int kb_begin = ks * ksteps / ksplit, kb_end = (ks + 1) * ksteps / ksplit;
             const CUtensorMap* tA = ti.special ? &args.tmA1 : &args.tmA0;
             const CUtensorMap* tB = ti.special ? args.tmB1 : args.tmB0;
             const int a_base = ti.special ? 0 : ti.seg * args.a_seg_stride;
             const uint64_t pw = ti.special ? pol_ws : pol_w;
             const bool gather =
-                C::kSwiGLU && !FP8 && args.gather_tok != nullptr && !ti.special;
+                C::kSwiGLU && !FP8 && !PAIR && args.gather_tok != nullptr && !ti.special;
+            // token rows this CTA loads (PAIR: its half of the tile's columns)
+            const int b_rows = PAIR ? ti.n_mma / 2 : ti.n_mma;
+            const int b_row0 = ti.b_row + (PAIR ? static_cast<int>(rank) * b_rows : 0);
             if (gather) {
                 __syncwarp();  // the previous tile's rows are all issued
                 for (int i = lane; i < ti.n_mma; i += 32)
                     s_gtok[i] = i < ti.n_valid ? __ldg(args.gather_tok + ti.b_row + i) : -1;
                 __syncwarp();
             }
-            const uint32_t bytes = C::kABytes + (gather ? 0 : ti.n_mma * 128);
+            // expected bytes (PAIR: the leader expects both CTAs' copies)
+            const uint32_t bytes =
+                PAIR ? 2u * (C::kABytes + b_rows * 128) : C::kABytes + (gather ? 0 : ti.n_mma * 128);
             for (int kb = kb_begin; kb < kb_end; ++kb) {
                 int got = 1;
                 if (lane == 0) got = ptx::mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag);
@@ -392,34 +422,46 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
                     __syncwarp();  // every lane's arrival is counted before lane 0 arrives
                 }
                 if (lane == 0) {
-                    ptx::mbar_arrive_expect_tx(&full_bar[stage], bytes);
-                    armed |= 1u << stage;
-                    armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+                    // completion is counted on this CTA's barrier, or (PAIR) on
+                    // the leader's, which alone expects the bytes
+                    uint32_t bar = ptx::smem_u32(&full_bar[stage]);
+                    if constexpr (PAIR) bar = ptx::mapa_shared(bar, 0);
+                    if (!PAIR || rank == 0) {
+                        ptx::mbar_arrive_expect_tx(&full_bar[stage], bytes);
+                        armed |= 1u << stage;
+                        armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+                    }
+                    auto load2d = [&](void* dst, const CUtensorMap* m, int c0, int c1,
+                                      uint64_t pol) {
+                        if constexpr (PAIR) ptx::tma_load_2d_pair(dst, m, c0, c1, bar, pol);
+                        else ptx::tma_load_2d(dst, m, c0, c1, &full_bar[stage], pol);
+                    };
+                    auto load3d = [&](void* dst, const CUtensorMap* m, int c0, int c1, int c2,
+                                      uint64_t pol) {
+                        if constexpr (PAIR) ptx::tma_load_3d_pair(dst, m, c0, c1, c2, bar, pol);
+                        else ptx::tma_load_3d(dst, m, c0, c1, c2, &full_bar[stage], pol);
+                    };
                     if constexpr (C::kDown) {
                         // MN-major A: one 3D copy of the tile's 128-byte-wide H
                         // chunks (bf16: 2*MB chunks of 64 values x 64 K-rows;
                         // FP8: MB chunks of 128 values x 128 K-rows), chunk-major
-                        ptx::tma_load_3d(sA, tA, 0, a_base + args.a_off0 + k0,
-                                         ti.blk * (FP8 ? MB : 2 * MB), &full_bar[stage], pw);
+                        load3d(sA, tA, 0, a_base + args.a_off0 + k0, ti.blk * (FP8 ? MB : 2 * MB),
+                               pw);
                     } else if constexpr (C::kSwiGLU) {
                         // gate and up tiles (adjacent matrices) in one 3D copy
-                        ptx::tma_load_3d(sA, tA, k0, ti.blk * 128, a_base + args.a_off0,
-                                         &full_bar[stage], pw);
+                        load3d(sA, tA, k0, ti.blk * 128, a_base + args.a_off0, pw);
                     } else if constexpr (MB == 2) {
                         // both 128-row blocks in one 256-row box
-                        ptx::tma_load_2d(sA, tA, k0, a_base + args.a_off0 + ti.blk * 256,
-                                         &full_bar[stage], pw);
+                        load2d(sA, tA, k0, a_base + args.a_off0 + ti.blk * 256, pw);
                     } else {
-                        ptx::tma_load_2d(sA, tA, k0, a_base + args.a_off0 + ti.blk * 128,
-                                         &full_bar[stage], pw);
+                        load2d(sA, tA, k0, a_base + args.a_off0 + ti.blk * 128, pw);
                     }
                     if (!gather) {
                         int q = 0;
 #pragma unroll
                         for (int j = kNumBoxSizes - 1; j >= 0; --j) {
-                            if ((ti.n_mma >> 4) & (1 << j)) {
-                                ptx::tma_load_2d(sB + q * 128, &tB[j], k0, ti.b_row + q,
-                                                 &full_bar[stage], pol_x);
+                            if ((b_rows >> 4) & (1 << j)) {
+                                load2d(sB + q * 128, &tB[j], k0, b_row0 + q, pol_x);
                                 q += 16 << j;
                             }
                         }
@@ -443,7 +485,8 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // (PAIR: the leader only; its cta_group::2 MMAs span both CTAs)
+        if (lane == 0 && rank == 0) {
             uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
             bool ok = true;
             constexpr uint32_t kAMajor = C::kDown ? 1u : 0u;
@@ -452,10 +495,21 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
             // 128-row sub-tile) -- unused for FP8, where one chunk is 128 rows
             constexpr uint32_t kMnStep = FP8 ? 4096u : 2048u;
             constexpr uint32_t kMnLbo = FP8 ? 16384u : 8192u;
-            for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
+            // PAIR: arrive on the barrier at the same offset in both CTAs
+            auto commit = [&](uint64_t* bar) {
+                if constexpr (PAIR) {
+                    const uint32_t own = ptx::smem_u32(bar);
+                    ptx::mma_commit_pair(own);
+                    ptx::mma_commit_pair(ptx::mapa_shared(own, 1));
+                } else {
+                    ptx::mma_commit(bar);
+                }
+            };
+            constexpr uint32_t kM = PAIR ? 256u : 128u;
+            for (int t = unit; ok && t < total_tiles; t += units) {
                 TileInfo ti;
                 const int ks = t % ksplit;
-                if (!decode_tile(t / ksplit, nblk, nseg, ss, args.special_seg, ti)) continue;
+                if (!decode(t, ti)) continue;
                 const int kb_begin = ks * ksteps / ksplit, kb_end = (ks + 1) * ksteps / ksplit;
                 if (!ptx::mbar_wait(&acce_bar[acc], acc_phase ^ 1, abort_flag)) {
                     fail(DEV_ERR_TIMEOUT);
@@ -463,8 +517,8 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
                 }
                 ptx::tc_fence_after();
                 const uint32_t d0 = tmem_base + acc * C::kAccCols;
-                const uint32_t idesc = FP8 ? ptx::idesc_e4m3_f32(128, ti.n_mma, kAMajor, 0)
-                                           : ptx::idesc_bf16_f32(128, ti.n_mma, kAMajor, 0);
+                const uint32_t idesc = FP8 ? ptx::idesc_e4m3_f32(kM, ti.n_mma, kAMajor, 0)
+                                           : ptx::idesc_bf16_f32(kM, ti.n_mma, kAMajor, 0);
                 for (int kb = kb_begin; kb < kb_end; ++kb) {
                     if (!ptx::mbar_wait(&full_bar[stage], phase, abort_flag)) {
                         fail(DEV_ERR_TIMEOUT);
@@ -487,25 +541,28 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
                             const uint64_t adesc =
                                 C::kDown ? ptx::smem_desc_sw128(a_sub + kk * kMnStep, kMnLbo, 1024)
                                          : ptx::smem_desc_sw128(a_sub + kk * 32, 16, 1024);
-                            if constexpr (FP8) ptx::mma_fp8(d0 + j * NMAX, adesc, bdesc, idesc, accum);
-                            else ptx::mma_bf16(d0 + j * NMAX, adesc, bdesc, idesc, accum);
+                            if constexpr (FP8)
+                                ptx::mma_fp8<CG>(d0 + j * NMAX, adesc, bdesc, idesc, accum);
+                            else
+                                ptx::mma_bf16<CG>(d0 + j * NMAX, adesc, bdesc, idesc, accum);
                         }
                     }
-                    ptx::mma_commit(&empty_bar[stage]);
+                    commit(&empty_bar[stage]);
                     if (++stage == C::kStages) {
                         stage = 0;
                         phase ^= 1;
                     }
                 }
                 if (!ok) break;
-                ptx::mma_commit(&accf_bar[acc]);
+                commit(&accf_bar[acc]);
                 if (++acc == C::kAccStages) {
                     acc = 0;
                     acc_phase ^= 1;
                 }
             }
             // all issued MMAs must retire before TMEM is released
-            ptx::mma_commit(final_bar);
+            if constexpr (PAIR) ptx::mma_commit_pair(ptx::smem_u32(final_bar));
+            else ptx::mma_commit(final_bar);
             ptx::mbar_wait(final_bar, 0, nullptr);
         }
     } else {
@@ -515,10 +572,10 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
         const int row_in_tile = quarter * 32 + lane;
         uint32_t acc = 0, acc_phase = 0;
         uint32_t mi = 0, meta_phase = 0;
-        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+        for (int t = unit; t < total_tiles; t += units) {
             TileInfo ti;
             const int ks = t % ksplit;
-            if (!decode_tile(t / ksplit, nblk, nseg, ss, args.special_seg, ti)) continue;
+            if (!decode(t, ti)) continue;
             int32_t* w_tok = reinterpret_cast<int32_t*>(s_meta) + mi * 2 * NMAX;
             float* w_wt = reinterpret_cast<float*>(w_tok + NMAX);
             if constexpr (C::kMeta) {
@@ -728,7 +785,11 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
             }
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&acce_bar[acc]);
+            if (lane == 0) {
+                // PAIR: the accumulator buffer is free once both CTAs drained it
+                if constexpr (PAIR) ptx::mbar_arrive_cluster(ptx::mapa_shared(ptx::smem_u32(&acce_bar[acc]), 0));
+                else ptx::mbar_arrive(&acce_bar[acc]);
+            }
             if (++acc == C::kAccStages) {
                 acc = 0;
                 acc_phase ^= 1;
@@ -737,9 +798,12 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
     }
 
     ptx::tc_fence_before();
-    __syncthreads();
+    // PAIR: neither CTA leaves (or frees TMEM) while the other may still signal
+    // its barriers or the leader's MMAs may still write its TMEM
+    if constexpr (PAIR) ptx::cluster_sync();
+    else __syncthreads();
     ptx::tc_fence_after();
-    if (warp == 1) ptx::tmem_dealloc(tmem_base, C::kTmemCols);
+    if (warp == 1) ptx::tmem_dealloc<CG>(tmem_base, C::kTmemCols);
 }
 
 }  // namespace moe

@@ -393,34 +393,103 @@ T* at(void* ws, size_t off) {
 
 // ------------------------------------------------------------------ GEMM launch
 
-template <int EPI, int NMAX, int MB, bool FP8 = false>
+// Clusters of two CTAs (one per SM) of `kern` that can be resident at once.
+template <typename K>
+int resident_pairs(K kern, int threads, int smem) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) {
+        cudaGetLastError();
+        return 0;
+    }
+    return n;
+}
+
+template <int EPI, int NMAX, int MB, bool FP8 = false, bool PAIR = false>
 int32_t launch_gemm_n(const GemmArgs& a, int grid, cudaStream_t s, const char* name) {
-    using C = GemmCfg<EPI, NMAX, MB, FP8>;
+    using C = GemmCfg<EPI, NMAX, MB, FP8, PAIR>;
+    auto kern = grouped_gemm_kernel<EPI, NMAX, MB, FP8, PAIR>;
     int dev = 0;
     cudaGetDevice(&dev);
     static std::atomic<uint64_t> configured{0};
+    static std::atomic<int> pairs[64];
     const uint64_t bit = (dev < 64) ? (1ull << dev) : 0;
     if (!bit || !(configured.load() & bit)) {
-        if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI, NMAX, MB, FP8>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::kSmemBytes) != cudaSuccess)
             return MOE_ERR_CUDA;
+        if constexpr (PAIR) {
+            const int n = resident_pairs(kern, C::kThreads, C::kSmemBytes);
+            if (n < 1) return MOE_ERR_CUDA;
+            if (bit) pairs[dev].store(n);
+        }
         configured.fetch_or(bit);
     }
-    MOE_LAUNCH(name, s,
-               grouped_gemm_kernel<EPI, NMAX, MB, FP8><<<grid, C::kThreads, C::kSmemBytes, s>>>(a));
+    if constexpr (PAIR) {
+        // one cluster per pair tile (a tile = two adjacent CTA tiles), at most
+        // as many clusters as can be resident together (persistent grid)
+        const int n = bit ? pairs[dev].load() : resident_pairs(kern, C::kThreads, C::kSmemBytes);
+        if (n < 1) return MOE_ERR_CUDA;
+        const int clusters = std::max(1, std::min(n, (grid + 1) / 2));
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * clusters);
+        cfg.blockDim = dim3(C::kThreads);
+        cfg.dynamicSmemBytes = C::kSmemBytes;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        MOE_LAUNCH(name, s, if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return MOE_ERR_CUDA);
+    } else {
+        MOE_LAUNCH(name, s, kern<<<grid, C::kThreads, C::kSmemBytes, s>>>(a));
+    }
     return MOE_OK;
 }
 
+// MOE_PAIR=1 runs the expert GEMMs as CTA pairs (cta_group::2, M = 256 per
+// MMA, each CTA loading half of the token tile) for tiles of 64 or more token
+// rows.  Off by default: the pairs halve the token-tile reads from L2 but
+// measured slower at the Hy4 prefill shapes (the two CTAs advance in
+// lockstep), and only about 1% faster on the tensor-bound skewed batch.
+bool use_pair() {
+    static const bool v = env_int("MOE_PAIR", 0) != 0;
+    return v;
+}
+
 template <int EPI, int MB, bool FP8 = false>
-int32_t launch_gemm_mb(int nmax, const GemmArgs& a, int grid, cudaStream_t s, const char* name) {
+int32_t launch_gemm_mb(int nmax, const GemmArgs& a, int grid, cudaStream_t s, const char* name,
+                       bool pair = false) {
     switch (nmax) {
         case 16: return launch_gemm_n<EPI, 16, MB, FP8>(a, grid, s, name);
         case 32: return launch_gemm_n<EPI, 32, MB, FP8>(a, grid, s, name);
-        case 64: return launch_gemm_n<EPI, 64, MB, FP8>(a, grid, s, name);
-        case 128: return launch_gemm_n<EPI, 128, MB, FP8>(a, grid, s, name);
-        case 160: return launch_gemm_n<EPI, 160, MB, FP8>(a, grid, s, name);
-        case 256: return launch_gemm_n<EPI, 256, MB, FP8>(a, grid, s, name);
+        case 64:
+            return pair ? launch_gemm_n<EPI, 64, MB, FP8, true>(a, grid, s, name)
+                        : launch_gemm_n<EPI, 64, MB, FP8>(a, grid, s, name);
+        case 128:
+            return pair ? launch_gemm_n<EPI, 128, MB, FP8, true>(a, grid, s, name)
+                        : launch_gemm_n<EPI, 128, MB, FP8>(a, grid, s, name);
+        case 160:
+            return pair ? launch_gemm_n<EPI, 160, MB, FP8, true>(a, grid, s, name)
+                        : launch_gemm_n<EPI, 160, MB, FP8>(a, grid, s, name);
+        case 256:
+            return pair ? launch_gemm_n<EPI, 256, MB, FP8, true>(a, grid, s, name)
+                        : launch_gemm_n<EPI, 256, MB, FP8>(a, grid, s, name);
         default: return MOE_ERR_UNSUPPORTED;
     }
 }
@@ -430,11 +499,12 @@ template <int EPI>
 int32_t launch_gemm_fp8(int nmax, int mb, const GemmArgs& a, int64_t max_tiles, cudaStream_t s,
                         const char* name) {
     int grid = static_cast<int>(std::min<int64_t>(sm_count(), std::max<int64_t>(1, max_tiles)));
+    const bool pair = use_pair() && nmax >= 64;
     if constexpr (EPI == EPI_SWIGLU) {
-        return launch_gemm_mb<EPI, 2, true>(nmax, a, grid, s, name);
+        return launch_gemm_mb<EPI, 2, true>(nmax, a, grid, s, name, pair);
     } else {
         static_assert(EPI == EPI_DOWN_STORE, "FP8 down GEMM uses the store epilogue");
-        if (mb == 2) return launch_gemm_mb<EPI, 2, true>(nmax, a, grid, s, name);
+        if (mb == 2) return launch_gemm_mb<EPI, 2, true>(nmax, a, grid, s, name, pair);
         return launch_gemm_mb<EPI, 1, true>(nmax, a, grid, s, name);
     }
 }
@@ -445,7 +515,8 @@ int32_t launch_gemm(int nmax, int mb, const GemmArgs& a, int64_t max_tiles, cuda
                     const char* name) {
     int grid = static_cast<int>(std::min<int64_t>(sm_count(), std::max<int64_t>(1, max_tiles)));
     if constexpr (EPI == EPI_SWIGLU) {
-        return launch_gemm_mb<EPI, 2>(nmax, a, grid, s, name);
+        const bool pair = use_pair() && nmax >= 64 && a.gather_tok == nullptr;
+        return launch_gemm_mb<EPI, 2>(nmax, a, grid, s, name, pair);
     } else if constexpr (EPI == EPI_LOGITS) {
         if (nmax == 256) {
             if (mb == 2) return launch_gemm_n<EPI, 256, 2>(a, grid, s, name);
@@ -459,7 +530,8 @@ int32_t launch_gemm(int nmax, int mb, const GemmArgs& a, int64_t max_tiles, cuda
         if (mb == 2) return launch_gemm_n<EPI, 32, 2>(a, grid, s, name);
         return launch_gemm_n<EPI, 32, 1>(a, grid, s, name);
     } else {
-        if (mb == 2) return launch_gemm_mb<EPI, 2>(nmax, a, grid, s, name);
+        const bool pair = EPI == EPI_DOWN_STORE && use_pair() && nmax >= 64 && mb == 2;
+        if (mb == 2) return launch_gemm_mb<EPI, 2>(nmax, a, grid, s, name, pair);
         return launch_gemm_mb<EPI, 1>(nmax, a, grid, s, name);
     }
 }
@@ -660,6 +732,23 @@ int32_t run_gather(const TIn* x, int64_t T, int H, int k, const int32_t* pos, in
     MOE_LAUNCH("dispatch_gather", s,
                gather_kernel<TIn, TOut><<<blocks, warps * 32, 0, s>>>(x, T, H, k, pos, n_rows,
                                                                       x_perm, x_bf16, acc_zero));
+    return MOE_OK;
+}
+
+// out[t] = sum over the token's rows of y (slot order, the shared row last),
+// one warp per (token, segment of H).
+template <typename TOut>
+int32_t run_gather_sum(const __nv_bfloat16* y, const int32_t* pos, int64_t T, int H, int k,
+                       int64_t n_rows, int64_t shared_row0, TOut* out, int32_t* status,
+                       cudaStream_t s) {
+    const int warps = 8;
+    const int64_t segs = (H / 8 + kSegVecs - 1) / kSegVecs;
+    const unsigned blocks = static_cast<unsigned>((T * segs + warps - 1) / warps);
+    // two rows' loads in flight per lane before adding: measured faster than
+    // wider batches, whose register use lowers the number of resident warps
+    MOE_LAUNCH("combine_gather", s,
+               (gather_sum_kernel<TOut, 2><<<blocks, warps * 32, 0, s>>>(
+                   y, pos, T, H, k, n_rows, shared_row0, out, status)));
     return MOE_OK;
 }
 
@@ -1042,24 +1131,12 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
         if (f32) return run_finalize<float>(out_acc, static_cast<float*>(out), T * H, s);
         return run_finalize<__nv_bfloat16>(out_acc, static_cast<__nv_bfloat16*>(out), T * H, s);
     }
-    {
-        const int warps = 8;
-        const int64_t segs = (p->H / 8 + kSegVecs - 1) / kSegVecs;
-        const unsigned blocks = static_cast<unsigned>((T * segs + warps - 1) / warps);
-        const int64_t shared_row0 = S ? T * k : -1;
-        if (f32) {
-            MOE_LAUNCH("combine_gather", s,
-                       gather_sum_kernel<float><<<blocks, warps * 32, 0, s>>>(
-                           y_perm, pos, T, p->H, p->top_k, T * k, shared_row0,
-                           static_cast<float*>(out), status));
-        } else {
-            MOE_LAUNCH("combine_gather", s,
-                       gather_sum_kernel<__nv_bfloat16><<<blocks, warps * 32, 0, s>>>(
-                           y_perm, pos, T, p->H, p->top_k, T * k, shared_row0,
-                           static_cast<__nv_bfloat16*>(out), status));
-        }
-    }
-    return MOE_OK;
+    const int64_t shared_row0 = S ? T * k : -1;
+    if (f32)
+        return run_gather_sum(y_perm, pos, T, p->H, p->top_k, T * k, shared_row0,
+                              static_cast<float*>(out), status, s);
+    return run_gather_sum(y_perm, pos, T, p->H, p->top_k, T * k, shared_row0,
+                          static_cast<__nv_bfloat16*>(out), status, s);
 }
 
 }  // extern "C"
@@ -1305,16 +1382,8 @@ int32_t moe_forward_fp8(const moe_problem* p, const void* x, const void* gate_w,
                                                 "expert_down_gemm_fp8"));
     }
     // 6. fixed-order combine into token order
-    {
-        const int warps = 8;
-        const int64_t segs = (H / 8 + kSegVecs - 1) / kSegVecs;
-        const unsigned blocks = static_cast<unsigned>((T * segs + warps - 1) / warps);
-        MOE_LAUNCH("combine_gather", s,
-                   gather_sum_kernel<__nv_bfloat16><<<blocks, warps * 32, 0, s>>>(
-                       y_perm, pos, T, p->H, p->top_k, T * k, S ? T * k : -1,
-                       static_cast<__nv_bfloat16*>(out), status));
-    }
-    return MOE_OK;
+    return run_gather_sum(y_perm, pos, T, p->H, p->top_k, T * k, S ? T * k : -1,
+                          static_cast<__nv_bfloat16*>(out), status, s);
 }
 
 int32_t moe_read_device_status(const void* ws, int32_t* status_out, void* stream) {

@@ -498,7 +498,7 @@ __global__ void combine_kernel(const T* __restrict__ y_perm, const int32_t* __re
 // row, so even a few tokens spread over many warps.
 constexpr int kSegVecs = 64;  // 16-byte vectors per warp segment
 
-template <typename TOut>
+template <typename TOut, int kBatch>
 __global__ void gather_sum_kernel(const __nv_bfloat16* __restrict__ y,
                                   const int32_t* __restrict__ pos, int64_t T, int H, int k,
                                   int64_t n_rows, int64_t shared_row0, TOut* __restrict__ out,
@@ -534,18 +534,27 @@ __global__ void gather_sum_kernel(const __nv_bfloat16* __restrict__ y,
                 acc[2 * e + 1] += f.y;
             }
         };
-#pragma unroll 4
-        for (int j = 0; j < k; ++j) {
-            const int r = __shfl_sync(0xffffffffu, my_pos, j);
-            if (r >= 0) {
-                if (oka) add8(acc_a, yv[r * row_vecs + va]);
-                if (okb) add8(acc_b, yv[r * row_vecs + vb]);
+        // rows in slot order (the shared expert's last), loaded kBatch at a
+        // time before any is added; the additions stay in slot order
+        const int n_rows_t = k + (shared_row0 >= 0 ? 1 : 0);
+        for (int j0 = 0; j0 < n_rows_t; j0 += kBatch) {
+            uint4 qa[kBatch], qb[kBatch];
+            bool has[kBatch];
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b) {
+                const int j = j0 + b;
+                int64_t r = -1;
+                if (j < k) r = __shfl_sync(0xffffffffu, my_pos, j & 31);
+                else if (j < n_rows_t) r = shared_row0 + t;
+                has[b] = r >= 0;
+                if (has[b] && oka) qa[b] = yv[r * row_vecs + va];
+                if (has[b] && okb) qb[b] = yv[r * row_vecs + vb];
             }
-        }
-        if (shared_row0 >= 0) {
-            const int64_t r = shared_row0 + t;
-            if (oka) add8(acc_a, yv[r * row_vecs + va]);
-            if (okb) add8(acc_b, yv[r * row_vecs + vb]);
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b) {
+                if (has[b] && oka) add8(acc_a, qa[b]);
+                if (has[b] && okb) add8(acc_b, qb[b]);
+            }
         }
         auto put = [&](const float (&acc)[8], int v) {
             if constexpr (sizeof(TOut) == 2) {

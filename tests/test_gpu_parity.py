@@ -349,3 +349,30 @@ def test_forward_gather_variants_agree():
         r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True,
                            text=True, env={**os.environ, **env}, timeout=600)
         assert r.returncode == 0 and "ok" in r.stdout, (env, r.stdout[-2000:], r.stderr[-2000:])
+
+
+def test_forward_cta_pair_variant():
+    """Expert GEMMs run as CTA pairs (MOE_PAIR=1: cta_group::2 MMAs of
+    M = 256, each CTA loading half of the token tile): bf16 layers with an odd
+    number of gate/up weight blocks (I = 384) and a ragged H (320), and the
+    FP8 layer, each against the oracle in a fresh process."""
+    import os
+    import subprocess
+    import sys
+    code = (
+        "import torch, sys; sys.path.insert(0, '.'); sys.path.insert(0, 'tests');"
+        "from test_gpu_parity import cfg, run_forward;"
+        "from parity_util import forward_parity, to_cpu_inputs;"
+        "from sparse_moe_layer_06_b200.workloads import make_inputs;"
+        "import test_gpu_fp8 as f8;"
+        "shapes = [dict(T=300, H=512, E=16, k=4, I=384), dict(T=200, H=320, E=12, k=3, I=192)];"
+        "[forward_parity(inp, c, *run_forward(c, inp)) for c, inp in "
+        "((c, make_inputs(c, seed=10, device='cuda')) for c in (cfg(**s) for s in shapes))];"
+        "inp = make_inputs(f8.SMALL, seed=3, device='cuda');"
+        "out, idx, w, _, _ = f8.run_fp8(f8.SMALL, inp);"
+        "f8.oracle_fp8_parity(f8.SMALL, to_cpu_inputs(inp), out, idx, w, list(range(f8.SMALL.T)));"
+        "print('ok')")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True,
+                       env={**os.environ, "MOE_PAIR": "1"}, timeout=600)
+    assert r.returncode == 0 and "ok" in r.stdout, (r.stdout[-2000:], r.stderr[-2000:])
