@@ -211,7 +211,7 @@ def whole_job_rate(units_per_rank: int, world: int, seconds: float) -> float:
 
 # ------------------------------------------------------------------ CPU oracle baseline
 
-def oracle_baseline(cfg, cpu_inp, budget_s=12.0, max_tokens=256):
+def oracle_baseline(cfg, cpu_inp, budget_s=12.0, max_tokens=2048):
     """Time the CPU oracle (as it stands) on a seeded token sample of the same
     workload: batches of tokens until ~budget_s of work.  Returns a dict."""
     import oracle
