@@ -620,15 +620,15 @@ int32_t run_logits(const moe_problem* p, const void* x, const void* gate_w, floa
 }
 
 // Top-k over the logits; n_parts > 1 sums that many [T,E] slices first (in
-// slice order) and leaves the sum in the first slice.
+// slice order), leaving the sum in the first slice when keep_sum is set.
 int32_t run_topk(const moe_problem* p, float* logits, const float* bias, int32_t* idx, float* w,
-                 cudaStream_t s, int n_parts = 1) {
+                 cudaStream_t s, int n_parts = 1, bool keep_sum = false) {
     const int warps = 8;
     const unsigned blocks = static_cast<unsigned>((p->T + warps - 1) / warps);
     MOE_LAUNCH("route_topk", s,
-               topk_kernel<<<blocks, warps * 32, 0, s>>>(logits, n_parts, p->T * p->E, bias, p->T,
-                                                         p->E, p->top_k, p->routed_scale, idx,
-                                                         w));
+               topk_kernel<<<blocks, warps * 32, 0, s>>>(logits, n_parts, p->T * p->E, keep_sum,
+                                                         bias, p->T, p->E, p->top_k,
+                                                         p->routed_scale, idx, w));
     return MOE_OK;
 }
 
@@ -1208,8 +1208,8 @@ int32_t moe_router_stats(const moe_problem* p, const void* x, const void* gate_w
     int32_t* counts = at<int32_t>(ws, L.counts);
     float* partial = at<float>(ws, L.partial);
     MOE_TRY(run_logits(p, x, gate_w, logits, status, s, true));
-    MOE_TRY(run_topk(p, logits, bias, idx, at<float>(ws, L.w), s,
-                     logits_plan(p, true).splits));
+    MOE_TRY(run_topk(p, logits, bias, idx, at<float>(ws, L.w), s, logits_plan(p, true).splits,
+                     true));
     if (cudaMemsetAsync(counts, 0, p->E * sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
     const int nblocks = static_cast<int>((p->T + kStatsTokensPerBlock - 1) / kStatsTokensPerBlock);
     MOE_LAUNCH("router_prob_partial", s,

@@ -41,29 +41,40 @@ __global__ void router_logits_f32_kernel(const float* __restrict__ x,
 // The renormalised weights are computed as the softmax over the k selected
 // logits, which equals p_j / sum_sel p (the full-softmax normaliser cancels).
 __global__ void topk_kernel(float* __restrict__ logits, int n_parts, int64_t part_stride,
-                            const float* __restrict__ bias, int64_t T, int E, int k, float scale,
-                            int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
+                            bool keep_sum, const float* __restrict__ bias, int64_t T, int E, int k,
+                            float scale, int32_t* __restrict__ idx_out,
+                            float* __restrict__ w_out) {
     const int lane = threadIdx.x & 31;
     const int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= T) return;
     constexpr int kPer = kMaxExperts / 32;
     float v[kPer];
     uint32_t taken = 0;
+    // partial sums of a K-split GEMM, added in slice order; all loads are
+    // issued before anything is stored, so they overlap
+    const float* row = logits + t * E;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = e < E ? row[e] : 0.0f;
+    }
+#pragma unroll 1
+    for (int q = 1; q < n_parts; ++q) {
+        const float* part = row + q * part_stride;
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E) v[i] += part[e];
+        }
+    }
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
         const int e = lane + 32 * i;
         if (e < E) {
-            // partial sums of a K-split GEMM: added in slice order, the total
-            // kept in the first slice for later readers
-            float l = logits[t * E + e];
-            if (n_parts > 1) {
-                for (int q = 1; q < n_parts; ++q) l += logits[q * part_stride + t * E + e];
-                logits[t * E + e] = l;
-            }
-            if (bias) l += bias[e];
-            v[i] = l;
+            // the summed logits kept in the first slice for later readers
+            if (n_parts > 1 && keep_sum) logits[t * E + e] = v[i];
+            if (bias) v[i] += bias[e];
         } else {
-            v[i] = 0.0f;
             taken |= 1u << i;
         }
     }

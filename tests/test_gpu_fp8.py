@@ -213,3 +213,31 @@ def test_forward_fp8_hy4_prefill_sampled(hy4):
                              tokens=toks, forced_idx=forced)
     got = out.float().cpu().numpy()[toks]
     assert_close_out(got, ref["out"], "hy4_prefill fp8 forward", OUT_TOL)
+
+
+def test_forward_fp8_hy4_decode_sampled(hy4):
+    """The Hy4-shape decode batch (T=64: about two rows per touched expert,
+    the smallest token tiles) with FP8 weights; the oracle checks a seeded
+    sample of tokens on the experts they reach."""
+    c, inp = hy4
+    cd = CONFIGS["hy4_decode"]
+    out, idx, w, gq, _ = run_fp8(cd, inp, T=cd.T)
+    cpu = to_cpu_inputs({k: v for k, v in inp.items() if k != "expert_w"})
+    cpu["x"] = cpu["x"][:cd.T]
+    orc = oracle.route(cpu["x"], cpu["gate_w"], cd.top_k, cd.routed_scale,
+                       logit_bias=cpu["logit_bias"])
+    check_routing(idx.cpu().numpy(), w.cpu().numpy(), orc, cd.top_k)
+    toks = sample_tokens(cd.T, 4, seed=5)
+    gi = idx.cpu().numpy()[toks]
+    sel = sorted(set(int(e) for e in gi.ravel()))
+    rq, rs_gu, rs_d = oracle.quantize_weights_fp8(inp["expert_w"][sel].cpu())
+    assert_same_codes(tuple(t[sel] for t in gq), (rq, rs_gu, rs_d), "hy4 decode experts")
+    remap = {e: j for j, e in enumerate(sel)}
+    forced = np.vectorize(remap.get)(gi).astype(np.int32)
+    bias = cpu["logit_bias"][sel] if cpu["logit_bias"] is not None else None
+    sq, ss_gu, ss_d = oracle.quantize_weights_fp8(cpu["shared_w"].unsqueeze(0))
+    ref = oracle.forward_fp8(cpu["x"], cpu["gate_w"][sel], rq, rs_gu, rs_d, sq, ss_gu, ss_d,
+                             cd.top_k, cd.routed_scale, cd.clip_limit, logit_bias=bias,
+                             tokens=toks, forced_idx=forced)
+    got = out.float().cpu().numpy()[toks]
+    assert_close_out(got, ref["out"], "hy4_decode fp8 forward", OUT_TOL)

@@ -243,6 +243,8 @@ def test_combine_matches_oracle(dtype, S):
     dict(T=130, H=256, E=8, k=8, I=128),            # k == E
     dict(T=200, H=320, E=12, k=3, I=192),           # H, I not multiples of 128
     dict(T=64, H=256, E=16, k=2, I=128, S=0, scale=1.0, clip=0.0),  # no shared, no clip
+    dict(T=50, H=64, E=1, k=1, I=64),               # one expert, smallest H and I
+    dict(T=77, H=192, E=256, k=8, I=64),            # widest router, I below one tile
 ])
 def test_forward_matches_oracle(shape):
     c = cfg(**shape)
