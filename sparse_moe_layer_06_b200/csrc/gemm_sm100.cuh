@@ -40,6 +40,7 @@
 #include <cstdint>
 
 #include "ptx.cuh"
+#include "route_topk.cuh"
 
 namespace moe {
 
@@ -119,6 +120,18 @@ struct GemmArgs {
     // tile each; part s writes its partial sums at out + s * split_stride
     int32_t k_splits;
     int64_t split_stride;
+    // EPI_LOGITS, fused routing (route_idx set; one tile per CTA, all CTAs
+    // resident: a cooperative launch): after writing its partial logits each
+    // CTA counts itself in on route_count[chunk], waits (bounded) until all
+    // k_splits parts of its token chunk are written, and then routes its share
+    // of the chunk's tokens (softmax, top-k, renormalised weights x scale)
+    int32_t* route_idx;
+    float* route_w;
+    const float* route_bias;
+    int32_t* route_count;
+    int32_t route_k;
+    float route_scale;
+    int32_t route_keep_sum;
     // EPI_SWIGLU row gather: when gather_tok != nullptr, ordinary segments
     // take their token rows straight from gather_src ([n_tokens, K] bf16) at
     // rows gather_tok[b_row + i] instead of from tmB0 (the permuted copy)
@@ -189,6 +202,9 @@ struct GemmCfg {
     static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
     static_assert(kStages >= 2, "pipeline depth");
     static constexpr int kSmemBytes = kStages * kStageBytes + kTailBytes;
+    // barrier area: full/empty per stage, accumulator full/empty x2, final,
+    // metadata x2 (8 bytes each), then the TMEM slot and two flags
+    static_assert((2 * kStages + 7) * 8 + 3 * 4 <= kBarrierBytes, "barrier area");
     static constexpr int kThreads = 32 * (2 + kEpiWarps);
 };
 
@@ -263,6 +279,7 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
     uint64_t* metaf_bar = final_bar + 1;  // EPI_DOWN_ATOMIC column metadata ready (x2)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(metaf_bar + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* route_go = abort_flag + 1;  // EPI_LOGITS fused routing: the chunk is complete
     int32_t* s_sched = reinterpret_cast<int32_t*>(tail + C::kBarrierBytes);
     uint8_t* s_meta = tail + C::kBarrierBytes + C::kSchedBytes;
     int32_t* s_gtok = reinterpret_cast<int32_t*>(s_meta + C::kMetaBytes);
@@ -804,6 +821,44 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
     else __syncthreads();
     ptx::tc_fence_after();
     if (warp == 1) ptx::tmem_dealloc<CG>(tmem_base, C::kTmemCols);
+
+    if constexpr (EPI == EPI_LOGITS) {
+        if (args.route_idx != nullptr) {
+            // fused routing: this CTA ran exactly tile blockIdx.x (nblk == 1)
+            const int ks = static_cast<int>(blockIdx.x) % ksplit;
+            const int chunk = static_cast<int>(blockIdx.x) / ksplit;
+            __threadfence();  // this CTA's partial logits, before the count below
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                atomicAdd(args.route_count + chunk, 1);
+                int go = 0;
+                const uint64_t t0 = clock64();
+                while (true) {
+                    if (ptx::ld_acquire_gpu(args.route_count + chunk) >= ksplit) {
+                        go = 1;
+                        break;
+                    }
+                    if (static_cast<uint64_t>(clock64()) - t0 > ptx::kMaxWaitCycles) break;
+                    __nanosleep(128);
+                }
+                if (!go) set_device_error(args.status, DEV_ERR_TIMEOUT);
+                *route_go = go;
+            }
+            __syncthreads();
+            if (*route_go) {
+                const int cl = args.single_chunk_len;
+                const int64_t r0 = static_cast<int64_t>(chunk) * cl;
+                const int64_t rows = min(static_cast<int64_t>(cl), args.single_rows - r0);
+                const int64_t share = (rows + ksplit - 1) / ksplit;
+                const int64_t a = r0 + ks * share;
+                const int64_t b = min(r0 + rows, a + share);
+                for (int64_t t = a + warp; t < b; t += blockDim.x >> 5)
+                    route_one_token(reinterpret_cast<float*>(args.out), ksplit, args.split_stride,
+                                    args.route_keep_sum != 0, args.route_bias, t, args.M_total,
+                                    args.route_k, args.route_scale, args.route_idx, args.route_w);
+            }
+        }
+    }
 }
 
 }  // namespace moe

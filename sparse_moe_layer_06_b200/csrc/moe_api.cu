@@ -282,6 +282,12 @@ LogitsPlan logits_plan(const moe_problem* p, bool allow_split) {
 }
 
 
+// Token chunks of the router GEMM (one routing counter each).
+int64_t logits_chunks(const moe_problem* p) {
+    const LogitsPlan lp = logits_plan(p, true);
+    return std::max<int64_t>(1, (p->T + lp.nmax - 1) / lp.nmax);
+}
+
 // ------------------------------------------------------------------ workspace layout
 
 struct Carve {
@@ -294,7 +300,8 @@ struct Carve {
 };
 
 struct Layout {
-    size_t status, logits, idx, w, hist, base, counts, offsets, partial, sched_gu, sched_dn, pos, src, row_w;
+    size_t status, logits, rcount, idx, w, hist, base, counts, offsets, partial, sched_gu, sched_dn,
+        pos, src, row_w;
     size_t x_perm, x_bf16, w_bf16, ws_bf16, h_perm, out_acc, y_perm, x_q, s_x, total;
 };
 
@@ -312,6 +319,7 @@ Layout layout_for(const moe_problem* p, int call, int64_t ffn_rows = 0, int ffn_
             break;
         case MOE_CALL_ROUTE:
             L.logits = c.take(logits_plan(p, true).splits * T * E * 4);
+            L.rcount = c.take(logits_chunks(p) * 4);
             break;
         case MOE_CALL_PERMUTE:
             L.hist = c.take(perm_chunks(T) * E * 4);
@@ -331,6 +339,7 @@ Layout layout_for(const moe_problem* p, int call, int64_t ffn_rows = 0, int ffn_
             break;
         case MOE_CALL_ROUTER_STATS:
             L.logits = c.take(logits_plan(p, true).splits * T * E * 4);
+            L.rcount = c.take(logits_chunks(p) * 4);
             L.idx = c.take(T * k * 4);
             L.w = c.take(T * k * 4);
             L.partial = c.take(((T + kStatsTokensPerBlock - 1) / kStatsTokensPerBlock) * E * 4);
@@ -338,6 +347,7 @@ Layout layout_for(const moe_problem* p, int call, int64_t ffn_rows = 0, int ffn_
             break;
         case MOE_CALL_FORWARD_FP8:
             L.logits = c.take(logits_plan(p, true).splits * T * E * 4);
+            L.rcount = c.take(logits_chunks(p) * 4);
             L.idx = c.take(T * k * 4);
             L.w = c.take(T * k * 4);
             L.hist = c.take(perm_chunks(T) * E * 4);
@@ -358,6 +368,7 @@ Layout layout_for(const moe_problem* p, int call, int64_t ffn_rows = 0, int ffn_
         case MOE_CALL_FORWARD:
         default:
             L.logits = c.take(logits_plan(p, true).splits * T * E * 4);
+            L.rcount = c.take(logits_chunks(p) * 4);
             L.idx = c.take(T * k * 4);
             L.w = c.take(T * k * 4);
             L.hist = c.take(perm_chunks(T) * E * 4);
@@ -418,7 +429,8 @@ int resident_pairs(K kern, int threads, int smem) {
 }
 
 template <int EPI, int NMAX, int MB, bool FP8 = false, bool PAIR = false>
-int32_t launch_gemm_n(const GemmArgs& a, int grid, cudaStream_t s, const char* name) {
+int32_t launch_gemm_n(const GemmArgs& a, int grid, cudaStream_t s, const char* name,
+                      bool coop = false) {
     using C = GemmCfg<EPI, NMAX, MB, FP8, PAIR>;
     auto kern = grouped_gemm_kernel<EPI, NMAX, MB, FP8, PAIR>;
     int dev = 0;
@@ -453,6 +465,19 @@ int32_t launch_gemm_n(const GemmArgs& a, int grid, cudaStream_t s, const char* n
         attr[0].val.clusterDim.x = 2;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        MOE_LAUNCH(name, s, if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return MOE_ERR_CUDA);
+    } else if (coop) {
+        // every CTA resident at once (the fused routing phase waits across CTAs)
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(C::kThreads);
+        cfg.dynamicSmemBytes = C::kSmemBytes;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         MOE_LAUNCH(name, s, if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return MOE_ERR_CUDA);
@@ -582,9 +607,26 @@ GemmArgs base_args(int32_t* status) {
     return a;
 }
 
-// Router logits through tcgen05 (bf16 x and gate weight).
+// Fused routing outputs of the router GEMM (see GemmArgs::route_idx).
+struct RouteOut {
+    const float* bias;
+    int32_t* idx;
+    float* w;
+    int32_t* count;  // logits_chunks(p) counters, zeroed here
+    bool keep_sum;
+};
+
+// MOE_FUSED_ROUTE=0 keeps the router GEMM and the top-k kernel separate.
+bool fused_route_enabled() {
+    static const bool v = env_int("MOE_FUSED_ROUTE", 1) != 0;
+    return v;
+}
+
+// Router logits through tcgen05 (bf16 x and gate weight); with `route`, the
+// same launch also routes every token (one tile per CTA, cooperative launch).
 int32_t run_logits_bf16(const moe_problem* p, const void* x, const void* gate_w, float* logits,
-                        int32_t* status, cudaStream_t s, const LogitsPlan& lp) {
+                        int32_t* status, cudaStream_t s, const LogitsPlan& lp,
+                        const RouteOut* route = nullptr) {
     GemmArgs a = base_args(status);
     if (!make_tmap(&a.tmA0, gate_w, p->E, p->H, 128 * lp.mb)) return MOE_ERR_CUDA;
     if (!make_tmap_rows(a.tmB0, x, p->T, p->H)) return MOE_ERR_CUDA;
@@ -600,6 +642,31 @@ int32_t run_logits_bf16(const moe_problem* p, const void* x, const void* gate_w,
     a.out_ld = p->E;
     a.k_splits = lp.splits;
     a.split_stride = p->T * static_cast<int64_t>(p->E);
+    if (route) {
+        const int64_t chunks = (p->T + lp.nmax - 1) / lp.nmax;
+        const int64_t tiles = chunks * lp.splits;  // one weight block: E <= 128 * mb
+        if (cudaMemsetAsync(route->count, 0, chunks * sizeof(int32_t), s) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        a.route_idx = route->idx;
+        a.route_w = route->w;
+        a.route_bias = route->bias;
+        a.route_count = route->count;
+        a.route_k = p->top_k;
+        a.route_scale = p->routed_scale;
+        a.route_keep_sum = route->keep_sum ? 1 : 0;
+        const int grid = static_cast<int>(tiles);
+        const char* name = "router_gemm_topk";
+        if (lp.nmax == 256) {
+            if (lp.mb == 2) return launch_gemm_n<EPI_LOGITS, 256, 2>(a, grid, s, name, true);
+            return launch_gemm_n<EPI_LOGITS, 256, 1>(a, grid, s, name, true);
+        }
+        if (lp.nmax == 64) {
+            if (lp.mb == 2) return launch_gemm_n<EPI_LOGITS, 64, 2>(a, grid, s, name, true);
+            return launch_gemm_n<EPI_LOGITS, 64, 1>(a, grid, s, name, true);
+        }
+        if (lp.mb == 2) return launch_gemm_n<EPI_LOGITS, 32, 2>(a, grid, s, name, true);
+        return launch_gemm_n<EPI_LOGITS, 32, 1>(a, grid, s, name, true);
+    }
     return launch_gemm<EPI_LOGITS>(
         lp.nmax, lp.mb, a, max_tiles(p->T, 1, lp.nmax, p->E, 128 * lp.mb) * lp.splits, s,
         "router_logits_gemm");
@@ -630,6 +697,24 @@ int32_t run_topk(const moe_problem* p, float* logits, const float* bias, int32_t
                                                          bias, p->T, p->E, p->top_k,
                                                          p->routed_scale, idx, w));
     return MOE_OK;
+}
+
+// Routing for the problem's own workspace: the fused router GEMM + top-k
+// launch (bf16, at most one tile per SM), else the K-split router GEMM and
+// the top-k kernel.  logits: logits_plan(p, true).splits [T,E] slices;
+// count: logits_chunks(p) ints.
+int32_t run_route(const moe_problem* p, const void* x, const void* gate_w, const float* bias,
+                  float* logits, int32_t* count, int32_t* idx, float* w, bool keep_sum,
+                  int32_t* status, cudaStream_t s) {
+    const LogitsPlan lp = logits_plan(p, true);
+    if (p->dtype == MOE_BF16 && fused_route_enabled() &&
+        logits_chunks(p) * lp.splits <= sm_count()) {
+        const RouteOut r{bias, idx, w, count, keep_sum};
+        return run_logits_bf16(p, x, gate_w, logits, status, s, lp, &r);
+    }
+    const int32_t rc = run_logits(p, x, gate_w, logits, status, s, true);
+    if (rc != MOE_OK) return rc;
+    return run_topk(p, logits, bias, idx, w, s, lp.splits, keep_sum);
 }
 
 int32_t run_cast(const void* in, void* out, int64_t n, cudaStream_t s) {
@@ -844,8 +929,8 @@ int32_t moe_route(const moe_problem* p, const void* x, const void* gate_w, const
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int32_t* status = at<int32_t>(ws, L.status);
     float* logits = at<float>(ws, L.logits);
-    MOE_TRY(run_logits(p, x, gate_w, logits, status, s, true));
-    return run_topk(p, logits, bias, topk_idx, topk_w, s, logits_plan(p, true).splits);
+    return run_route(p, x, gate_w, bias, logits, at<int32_t>(ws, L.rcount), topk_idx, topk_w,
+                     false, status, s);
 }
 
 int32_t moe_permute(const moe_problem* p, const int32_t* topk_idx, const void* x,
@@ -1018,8 +1103,8 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
     }
 
     // 1. route
-    MOE_TRY(run_logits(p, x, gate_w, logits, status, s, true));
-    MOE_TRY(run_topk(p, logits, bias, idx, w, s, logits_plan(p, true).splits));
+    MOE_TRY(run_route(p, x, gate_w, bias, logits, at<int32_t>(ws, L.rcount), idx, w, false,
+                      status, s));
 
     // 2. dispatch bookkeeping + schedules
     const int nmax = pick_nmax(static_cast<double>(T * k) / E);
@@ -1207,9 +1292,8 @@ int32_t moe_router_stats(const moe_problem* p, const void* x, const void* gate_w
     int32_t* idx = at<int32_t>(ws, L.idx);
     int32_t* counts = at<int32_t>(ws, L.counts);
     float* partial = at<float>(ws, L.partial);
-    MOE_TRY(run_logits(p, x, gate_w, logits, status, s, true));
-    MOE_TRY(run_topk(p, logits, bias, idx, at<float>(ws, L.w), s, logits_plan(p, true).splits,
-                     true));
+    MOE_TRY(run_route(p, x, gate_w, bias, logits, at<int32_t>(ws, L.rcount), idx,
+                      at<float>(ws, L.w), true, status, s));
     if (cudaMemsetAsync(counts, 0, p->E * sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
     const int nblocks = static_cast<int>((p->T + kStatsTokensPerBlock - 1) / kStatsTokensPerBlock);
     MOE_LAUNCH("router_prob_partial", s,
@@ -1283,9 +1367,8 @@ int32_t moe_forward_fp8(const moe_problem* p, const void* x, const void* gate_w,
     float* w = w_out ? w_out : at<float>(ws, L.w);
 
     // 1. route (bf16 gate GEMM, unquantized)
-    MOE_TRY(run_logits(p, x, gate_w, at<float>(ws, L.logits), status, s, true));
-    MOE_TRY(run_topk(p, at<float>(ws, L.logits), bias, idx, w, s,
-                     logits_plan(p, true).splits));
+    MOE_TRY(run_route(p, x, gate_w, bias, at<float>(ws, L.logits), at<int32_t>(ws, L.rcount), idx,
+                      w, false, status, s));
     // 2. dispatch
     const int nmax = pick_nmax(static_cast<double>(T * k) / E);
     const int nmax_dn = pick_down_nmax(nmax);

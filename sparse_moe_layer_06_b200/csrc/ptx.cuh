@@ -133,6 +133,13 @@ __device__ __forceinline__ void tma_load_3d_pair(void* smem_dst, const CUtensorM
         : "memory");
 }
 
+// Acquire load of a global counter (pairs with a release by another CTA).
+__device__ __forceinline__ int ld_acquire_gpu(const int32_t* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 // ---------------------------------------------------------------- clusters
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
