@@ -276,6 +276,20 @@ int32_t moe_forward_fp8(const moe_problem* problem, const void* x, const void* g
                         const float* shared_scale_d, void* out, int32_t* topk_idx_out,
                         float* topk_w_out, void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * moe_check_wait_timeout -- self-check of the bounded waits every kernel uses
+ * (mbarrier phase waits, and the global-counter wait of the fused routing
+ * step).  Launches one thread that waits on an mbarrier nobody arrives on and
+ * on a counter nobody increments, each with a limit of about 0.1 s; both give
+ * up, and MOE_ERR_TIMEOUT is written to the workspace's error word.
+ * *waits_timed_out (host) receives one bit per wait that gave up (3 = both).
+ * The workspace needs 256 bytes (any workspace from moe_workspace_size has
+ * them); the call waits for the stream.  Nothing faults or hangs, and the
+ * context stays usable: clear the error word with moe_clear_device_status.
+ */
+int32_t moe_check_wait_timeout(void* workspace, size_t ws_bytes, int32_t* waits_timed_out,
+                               void* stream);
+
 /* Copy the device error word of `workspace` to *status_out (host), waiting
  * for the stream.  Returns MOE_OK or MOE_ERR_CUDA / MOE_ERR_INVALID_ARG. */
 int32_t moe_read_device_status(const void* workspace, int32_t* status_out, void* stream);

@@ -831,16 +831,7 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
             __syncthreads();
             if (threadIdx.x == 0) {
                 atomicAdd(args.route_count + chunk, 1);
-                int go = 0;
-                const uint64_t t0 = clock64();
-                while (true) {
-                    if (ptx::ld_acquire_gpu(args.route_count + chunk) >= ksplit) {
-                        go = 1;
-                        break;
-                    }
-                    if (static_cast<uint64_t>(clock64()) - t0 > ptx::kMaxWaitCycles) break;
-                    __nanosleep(128);
-                }
+                const int go = ptx::wait_counter_at_least(args.route_count + chunk, ksplit) ? 1 : 0;
                 if (!go) set_device_error(args.status, DEV_ERR_TIMEOUT);
                 *route_go = go;
             }

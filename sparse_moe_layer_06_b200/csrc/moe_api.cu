@@ -1485,6 +1485,26 @@ int32_t moe_clear_device_status(void* ws, void* stream) {
     return MOE_OK;
 }
 
+int32_t moe_check_wait_timeout(void* ws, size_t ws_bytes, int32_t* waits_timed_out,
+                               void* stream) {
+    if (!ws || !waits_timed_out || ws_bytes < 256 || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    int32_t* status = reinterpret_cast<int32_t*>(base);
+    int32_t* counter = reinterpret_cast<int32_t*>(base + 64);
+    int32_t* result = reinterpret_cast<int32_t*>(base + 128);
+    if (cudaMemsetAsync(base + 64, 0, 128, s) != cudaSuccess) return MOE_ERR_CUDA;
+    // about 0.1 s per wait at the B200's clocks
+    const uint64_t limit = 200000000ull;
+    MOE_LAUNCH("wait_selftest", s,
+               wait_selftest_kernel<<<1, 32, 0, s>>>(counter, limit, status, result));
+    if (cudaMemcpyAsync(waits_timed_out, result, sizeof(int32_t), cudaMemcpyDeviceToHost, s) !=
+        cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
 int64_t moe_launch_count(void) { return g_launches.load(); }
 
 int32_t moe_profile_start(int32_t max_launches) {

@@ -65,7 +65,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
 // path is a bare try_wait; the cycle counter is only read between batches of
 // polls so that it never sits on the critical path of a completing phase.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          const volatile int* abort_flag) {
+                                          const volatile int* abort_flag,
+                                          uint64_t limit_cycles = kMaxWaitCycles) {
     const uint32_t addr = smem_u32(bar);
     if (mbar_try_wait(addr, parity)) return true;
     const uint64_t t0 = clock64();
@@ -75,7 +76,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
             if (mbar_try_wait(addr, parity)) return true;
         }
         if (abort_flag && *abort_flag) return false;
-        if (static_cast<uint64_t>(clock64()) - t0 > kMaxWaitCycles) return false;
+        if (static_cast<uint64_t>(clock64()) - t0 > limit_cycles) return false;
     }
 }
 
@@ -138,6 +139,19 @@ __device__ __forceinline__ int ld_acquire_gpu(const int32_t* p) {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
+}
+
+// Bounded wait (one thread) until the global counter at p reaches `target`
+// (another CTA's atomic add after a fence publishes its writes).  Returns
+// false if limit_cycles pass first.
+__device__ __forceinline__ bool wait_counter_at_least(const int32_t* p, int target,
+                                                      uint64_t limit_cycles = kMaxWaitCycles) {
+    const uint64_t t0 = clock64();
+    while (true) {
+        if (ld_acquire_gpu(p) >= target) return true;
+        if (static_cast<uint64_t>(clock64()) - t0 > limit_cycles) return false;
+        __nanosleep(128);
+    }
 }
 
 // ---------------------------------------------------------------- clusters

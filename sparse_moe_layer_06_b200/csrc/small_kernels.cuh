@@ -503,6 +503,30 @@ __global__ void gather_sum_kernel(const __nv_bfloat16* __restrict__ y,
     }
 }
 
+// ------------------------------------------------------------------ wait self-check
+
+// One thread runs the two bounded waits the kernels rely on against events
+// that never happen: an mbarrier nobody arrives on and a global counter nobody
+// increments.  Each gives up after limit_cycles and records MOE_ERR_TIMEOUT in
+// the error word; `result` gets one bit per wait that (correctly) gave up.
+__global__ void wait_selftest_kernel(const int32_t* counter, uint64_t limit_cycles,
+                                     int32_t* status, int32_t* result) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x != 0) return;
+    ptx::mbar_init(&bar, 1);
+    ptx::fence_mbar_init();
+    int bits = 0;
+    if (!ptx::mbar_wait(&bar, 0, nullptr, limit_cycles)) {
+        set_device_error(status, DEV_ERR_TIMEOUT);
+        bits |= 1;
+    }
+    if (!ptx::wait_counter_at_least(counter, 1, limit_cycles)) {
+        set_device_error(status, DEV_ERR_TIMEOUT);
+        bits |= 2;
+    }
+    *result = bits;
+}
+
 // ------------------------------------------------------------------ FP8 (E4M3) quantization
 //
 // Scales are powers of two, s = 2^n with n the smallest integer such that

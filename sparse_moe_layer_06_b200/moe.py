@@ -32,6 +32,7 @@ EXPORTED = (
     "moe_grouped_swiglu_ffn", "moe_combine", "moe_forward", "moe_read_device_status",
     "moe_clear_device_status", "moe_launch_count", "moe_profile_start", "moe_profile_stop",
     "moe_route_noalloc", "moe_router_stats", "moe_quantize_weights_fp8", "moe_forward_fp8",
+    "moe_check_wait_timeout",
 )
 ROUTE_NOALLOC_SCRATCH_BYTES = 1 << 20
 
@@ -115,6 +116,7 @@ def load_library(path: str = LIB_PATH):
             "moe_router_stats": (I32, [PP, P, P, P, P, P, P, P, P, ctypes.c_float, P, SZ, P]),
             "moe_quantize_weights_fp8": (I32, [PP, I32, P, P, P, P, P]),
             "moe_forward_fp8": (I32, [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]),
+            "moe_check_wait_timeout": (I32, [P, SZ, ctypes.POINTER(I32), P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -239,6 +241,16 @@ def moe_forward_fp8(problem, x, gate_w, logit_bias, expert_q, expert_s_gu, exper
         _ptr(topk_idx_out, torch.int32, "topk_idx_out", optional=True),
         _ptr(topk_w_out, torch.float32, "topk_w_out", optional=True),
         _ptr(workspace, None, "workspace"), workspace.numel(), _stream(stream)), "moe_forward_fp8")
+
+
+def moe_check_wait_timeout(workspace, stream=None) -> int:
+    """Run the bounded-wait self-check; returns the bits of the waits that gave
+    up (3 = both).  The workspace's error word is left at MOE_ERR_TIMEOUT."""
+    out = ctypes.c_int32(0)
+    _check(load_library().moe_check_wait_timeout(
+        _ptr(workspace, None, "workspace"), workspace.numel(), ctypes.byref(out),
+        _stream(stream)), "moe_check_wait_timeout")
+    return int(out.value)
 
 
 def moe_permute(problem, topk_idx, x, offsets, pos, src_token, x_perm, workspace, stream=None):
