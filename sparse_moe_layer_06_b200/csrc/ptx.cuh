@@ -112,7 +112,7 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
 // The same two loads for a CTA pair (cta_group::2): the copy lands in this
 // CTA's shared memory, its completion is counted on the mbarrier at the
 // shared::cluster address `bar_cluster`, which may belong to the peer CTA.
-// Plain (not multicast) tensor copies.
+// Plain tensor copies: one destination CTA each.
 __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* m, int32_t c0,
                                                  int32_t c1, uint32_t bar_cluster,
                                                  uint64_t policy) {
