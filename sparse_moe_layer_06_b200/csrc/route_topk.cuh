@@ -35,8 +35,26 @@ __device__ __forceinline__ void route_one_token(float* __restrict__ logits, int 
         const int e = lane + 32 * i;
         v[i] = e < E ? __ldcg(row + e) : 0.0f;
     }
+    // up to kMaxParts slices: every load issued before the first addition
+    constexpr int kMaxParts = 8;
+    float pv[kMaxParts - 1][kPer];
+#pragma unroll
+    for (int q = 1; q < kMaxParts; ++q) {
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int e = lane + 32 * i;
+            pv[q - 1][i] = (q < n_parts && e < E) ? __ldcg(row + q * part_stride + e) : 0.0f;
+        }
+    }
+#pragma unroll
+    for (int q = 1; q < kMaxParts; ++q) {
+        if (q < n_parts) {
+#pragma unroll
+            for (int i = 0; i < kPer; ++i) v[i] += pv[q - 1][i];
+        }
+    }
 #pragma unroll 1
-    for (int q = 1; q < n_parts; ++q) {
+    for (int q = kMaxParts; q < n_parts; ++q) {
         const float* part = row + q * part_stride;
 #pragma unroll
         for (int i = 0; i < kPer; ++i) {
