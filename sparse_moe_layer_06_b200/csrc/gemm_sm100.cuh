@@ -27,6 +27,13 @@
 // The accumulator is double-buffered in TMEM when it fits, so the epilogue of
 // tile i overlaps the main loop of tile i+1.
 //
+// Variants: FP8 (E4M3 operands, tcgen05.mma kind::f8f6f4, 128 K-values per
+// 128-byte row, scales applied in the epilogues); PAIR (two CTAs of a cluster
+// share a tile through cta_group::2 MMAs of M = 256, each holding its own
+// weight rows and half of the token rows); EPI_LOGITS with k_splits (the K
+// range split over several tiles into fp32 partial slices) and, optionally,
+// the routing of each token chunk once its parts are complete (route_idx).
+//
 // Operand layouts in shared memory (128-byte swizzle, 1024-byte atoms):
 //   K-major (x, h, gate/up weights): a tile row = 64 bf16 of K = 128 bytes;
 //     8 rows per atom; descriptor SBO = 1024 B; +32 B per K=16 step.
