@@ -201,7 +201,7 @@ struct GemmCfg {
     static constexpr int kMetaBytes = kMeta ? 2 * NMAX * 8 : 0;
     static constexpr int kEpiWarps = 8;
     // EPI_SWIGLU: token index of each row of the current tile (row gather)
-    static constexpr int kGatherBytes = kSwiGLU ? NMAX * 4 : 0;
+    static constexpr int kGatherBytes = kSwiGLU ? NMAX * 8 : 0;
     static constexpr int kTailBytes =
         1024 + kBarrierBytes + kSchedBytes + kMetaBytes + kGatherBytes;
     static constexpr int kMaxSmem = 227 * 1024;
@@ -289,7 +289,8 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
     volatile int* route_go = abort_flag + 1;  // EPI_LOGITS fused routing: the chunk is complete
     int32_t* s_sched = reinterpret_cast<int32_t*>(tail + C::kBarrierBytes);
     uint8_t* s_meta = tail + C::kBarrierBytes + C::kSchedBytes;
-    int32_t* s_gtok = reinterpret_cast<int32_t*>(s_meta + C::kMetaBytes);
+    // gathered tile: element offset of each row's token in the source
+    int64_t* s_goff = reinterpret_cast<int64_t*>(s_meta + C::kMetaBytes);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -410,8 +411,13 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
             const int b_row0 = ti.b_row + (PAIR ? static_cast<int>(rank) * b_rows : 0);
             if (gather) {
                 __syncwarp();  // the previous tile's rows are all issued
-                for (int i = lane; i < ti.n_mma; i += 32)
-                    s_gtok[i] = i < ti.n_valid ? __ldg(args.gather_tok + ti.b_row + i) : -1;
+                for (int i = lane; i < ti.n_mma; i += 32) {
+                    const int tok = i < ti.n_valid ? __ldg(args.gather_tok + ti.b_row + i) : -1;
+                    // padding rows (never stored) and out-of-range indices: a row of zeros
+                    s_goff[i] = static_cast<unsigned>(tok) < static_cast<unsigned>(args.n_tokens)
+                                    ? static_cast<int64_t>(tok) * args.K
+                                    : int64_t(-1);
+                }
                 __syncwarp();
             }
             // expected bytes (PAIR: the leader expects both CTAs' copies)
@@ -430,17 +436,23 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
                 uint8_t* sB = sA + C::kABytes;
                 const int k0 = kb * C::kKStep;
                 if (gather) {
+                    // lane: 16-byte chunk (lane & 7) of rows lane/8 + 4i; the
+                    // offsets of four rows are read before their copies are
+                    // issued (each copy is ordered against later loads)
                     const int chunk = lane & 7;
-                    for (int r = lane >> 3; r < ti.n_mma; r += 4) {
-                        int tok = s_gtok[r];
-                        if (static_cast<unsigned>(tok) >= static_cast<unsigned>(args.n_tokens))
-                            tok = -1;  // padding row, or an out-of-range index: zeros
-                        const void* src = tok >= 0
-                            ? static_cast<const void*>(gsrc + static_cast<size_t>(tok) * args.K +
-                                                       k0 + chunk * 8)
-                            : static_cast<const void*>(gsrc);
-                        ptx::cp_async_16(sB + r * 128 + ((chunk ^ (r & 7)) << 4), src,
-                                         tok >= 0 ? 16u : 0u);
+                    const bf16_raw_ptr base = gsrc + k0 + chunk * 8;
+                    for (int r0 = 0; r0 < ti.n_mma; r0 += 16) {  // n_mma: a multiple of 16
+                        int64_t off[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) off[j] = s_goff[r0 + (lane >> 3) + 4 * j];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int r = r0 + (lane >> 3) + 4 * j;
+                            ptx::cp_async_16(sB + r * 128 + ((chunk ^ (r & 7)) << 4),
+                                             off[j] >= 0 ? static_cast<const void*>(base + off[j])
+                                                         : static_cast<const void*>(gsrc),
+                                             off[j] >= 0 ? 16u : 0u);
+                        }
                     }
                     ptx::cp_async_mbar_arrive(&full_bar[stage]);
                     __syncwarp();  // every lane's arrival is counted before lane 0 arrives
