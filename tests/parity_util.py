@@ -12,12 +12,13 @@ import oracle
 OUT_TOL = 2e-2
 # Routing weights: w_j = scale * softmax(selected logits)_j, so a logit error
 # dl gives a relative weight error of at most 2*max|dl|.  The kernel's logits
-# are fp32 sums of H exact bf16 products (tensor-core accumulation); their
-# error grows like sqrt(H) * 2^-24 * |partial sums| and reaches ~6e-6 at
-# H=6144 (observed), so weights are checked to 1e-4 relative (about 8x the
-# largest error seen).  Near-tie band between the k-th and (k+1)-th
-# probability: 1e-5 relative (the stated routing rule).
-W_RTOL = 1e-4
+# are fp32 tensor-core sums of exact bf16 products over 8 K-slices of H/8,
+# added in slice order; over every token of the five named workloads the
+# largest weight error measured is 7.4e-6 (the skewed batch, whose logit bias
+# makes the logits largest), 1.0e-6 or less elsewhere, so weights are checked
+# to 1e-5 relative (the stated acceptance bound).  Near-tie band between the
+# k-th and (k+1)-th probability: 1e-5 relative (the stated routing rule).
+W_RTOL = 1e-5
 TIE_REL = 1e-5
 
 
