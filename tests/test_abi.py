@@ -137,3 +137,15 @@ def test_binding_refuses_cpu_tensors(lib):
     x = torch.zeros(4, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         moe.moe_router_logits(p, x, x, torch.zeros(4, 2), torch.zeros(256, dtype=torch.uint8))
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """Without the CUDA library there is nothing to fall back to: loading it
+    from a path where it does not exist raises, naming the build step."""
+    import importlib
+    fresh = importlib.reload(moe)  # a module instance with no library loaded yet
+    try:
+        with pytest.raises(RuntimeError, match="no non-CUDA implementation"):
+            fresh.load_library(str(tmp_path / "libmoe_b200.so"))
+    finally:
+        importlib.reload(moe)
