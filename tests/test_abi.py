@@ -149,3 +149,22 @@ def test_missing_library_fails_loudly(tmp_path):
             fresh.load_library(str(tmp_path / "libmoe_b200.so"))
     finally:
         importlib.reload(moe)
+
+
+def test_header_compiles_as_c_and_links(lib, tmp_path):
+    """A C99 program using include/moe.h links against the library and runs
+    its host-only calls (no GPU needed)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = os.path.join(ROOT, "tests", "c_api", "c_api_check.c")
+    exe = str(tmp_path / "c_api_check")
+    libdir = os.path.dirname(moe.LIB_PATH)
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        src, "-o", exe, "-L", libdir, "-lmoe_b200", f"-Wl,-rpath,{libdir}"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout + r.stderr
