@@ -164,7 +164,7 @@ struct GemmArgs {
 // The pipeline depth is whatever fits the 227 KB of shared memory.
 //   FP8   E4M3 operands (kind::f8f6f4): 128 K-elements per 128-byte row per
 //         stage instead of 64, scales applied in the epilogue
-template <int EPI, int NMAX, int MB, bool FP8 = false, bool PAIR = false>
+template <int EPI, int NMAX, int MB, bool FP8 = false, bool PAIR = false, int GW = 0>
 struct GemmCfg {
     static_assert(NMAX % 16 == 0 && NMAX >= 16 && NMAX <= 256, "N tile");
     static_assert(MB == 1 || MB == 2, "weight sub-tiles");
@@ -212,7 +212,10 @@ struct GemmCfg {
     // barrier area: full/empty per stage, accumulator full/empty x2, final,
     // metadata x2 (8 bytes each), then the TMEM slot and two flags
     static_assert((2 * kStages + 7) * 8 + 3 * 4 <= kBarrierBytes, "barrier area");
-    static constexpr int kThreads = 32 * (2 + kEpiWarps);
+    // GW > 0 (EPI_SWIGLU with the row gather): that many more warps copy the
+    // gathered token rows; the producer warp then only issues the weight copies
+    static_assert(GW == 0 || (EPI == EPI_SWIGLU && !FP8 && !PAIR), "gather warps");
+    static constexpr int kThreads = 32 * (2 + kEpiWarps + GW);
 };
 
 struct TileInfo {
@@ -269,9 +272,10 @@ __device__ __forceinline__ float clamp_keep_nan(float v, float lim) {
     return v > lim ? lim : (v < -lim ? -lim : v);
 }
 
-template <int EPI, int NMAX, int MB, bool FP8, bool PAIR>
-__global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs args) {
-    using C = GemmCfg<EPI, NMAX, MB, FP8, PAIR>;
+template <int EPI, int NMAX, int MB, bool FP8, bool PAIR, int GW>
+__global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ GemmArgs args) {
+    using C = GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>;
     constexpr int CG = PAIR ? 2 : 1;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned ring (the 128-byte swizzle atoms need it)
@@ -320,7 +324,8 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
     }
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
-            ptx::mbar_init(&full_bar[s], 1);
+            // GW > 0: one arrival of every gather lane per stage besides the producer's
+            ptx::mbar_init(&full_bar[s], 1 + 32 * GW);
             ptx::mbar_init(&empty_bar[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
@@ -406,10 +411,12 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
             const uint64_t pw = ti.special ? pol_ws : pol_w;
             const bool gather =
                 C::kSwiGLU && !FP8 && !PAIR && args.gather_tok != nullptr && !ti.special;
+            // GW > 0: the gather warps copy the rows; this warp only the weights
+            const bool own_gather = gather && GW == 0;
             // token rows this CTA loads (PAIR: its half of the tile's columns)
             const int b_rows = PAIR ? ti.n_mma / 2 : ti.n_mma;
             const int b_row0 = ti.b_row + (PAIR ? static_cast<int>(rank) * b_rows : 0);
-            if (gather) {
+            if (own_gather) {
                 __syncwarp();  // the previous tile's rows are all issued
                 for (int i = lane; i < ti.n_mma; i += 32) {
                     const int tok = i < ti.n_valid ? __ldg(args.gather_tok + ti.b_row + i) : -1;
@@ -423,6 +430,7 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
             // expected bytes (PAIR: the leader expects both CTAs' copies)
             const uint32_t bytes =
                 PAIR ? 2u * (C::kABytes + b_rows * 128) : C::kABytes + (gather ? 0 : ti.n_mma * 128);
+            // (gathered rows arrive through cp.async, counted as arrivals)
             for (int kb = kb_begin; kb < kb_end; ++kb) {
                 int got = 1;
                 if (lane == 0) got = ptx::mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag);
@@ -435,7 +443,7 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
                 uint8_t* sA = ring + stage * C::kStageBytes;
                 uint8_t* sB = sA + C::kABytes;
                 const int k0 = kb * C::kKStep;
-                if (gather) {
+                if (own_gather) {
                     // lane: 16-byte chunk (lane & 7) of rows lane/8 + 4i; the
                     // offsets of four rows are read before their copies are
                     // issued (each copy is ordered against later loads)
@@ -601,6 +609,73 @@ __global__ void __launch_bounds__(320, 1) grouped_gemm_kernel(const __grid_const
             else ptx::mma_commit(final_bar);
             ptx::mbar_wait(final_bar, 0, nullptr);
         }
+    } else if (GW > 0 && warp >= 2 + C::kEpiWarps) {
+        // ------------------------------------------------------------ row gather
+        // gather warp gw copies the 16-row groups gw, gw + GW, ... of each
+        // gathered tile (lane: 16-byte chunk lane & 7 of rows lane/8 + 4j of a
+        // group) and arrives once per stage on the full barrier, when its
+        // copies have landed (at once for tiles it has no rows of)
+        const int gw = warp - 2 - C::kEpiWarps;
+        const bf16_raw_ptr gsrc = reinterpret_cast<bf16_raw_ptr>(args.gather_src);
+        uint32_t stage = 0, phase = 0;
+        bool ok = true;
+        for (int t = unit; ok && t < total_tiles; t += units) {
+            TileInfo ti;
+            const int ks = t % ksplit;
+            if (!decode(t, ti)) continue;
+            const int kb_begin = ks * ksteps / ksplit, kb_end = (ks + 1) * ksteps / ksplit;
+            const bool gather = args.gather_tok != nullptr && !ti.special;
+            const int ngroups = ti.n_mma >> 4;
+            if (gather) {
+                __syncwarp();  // this warp's previous rows are all issued
+                for (int g = gw; g < ngroups; g += GW) {
+                    for (int i = lane; i < 16; i += 32) {
+                        const int r = g * 16 + i;
+                        const int tok =
+                            r < ti.n_valid ? __ldg(args.gather_tok + ti.b_row + r) : -1;
+                        s_goff[r] = static_cast<unsigned>(tok) <
+                                            static_cast<unsigned>(args.n_tokens)
+                                        ? static_cast<int64_t>(tok) * args.K
+                                        : int64_t(-1);
+                    }
+                }
+                __syncwarp();
+            }
+            for (int kb = kb_begin; kb < kb_end; ++kb) {
+                int got = 1;
+                if (lane == 0) got = ptx::mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag);
+                got = __shfl_sync(0xffffffffu, got, 0);
+                if (!got) {
+                    ok = false;
+                    break;
+                }
+                if (gather) {
+                    uint8_t* sB = ring + stage * C::kStageBytes + C::kABytes;
+                    const int chunk = lane & 7;
+                    const bf16_raw_ptr base = gsrc + kb * C::kKStep + chunk * 8;
+                    for (int g = gw; g < ngroups; g += GW) {
+                        const int r0 = g * 16;
+                        int64_t off[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) off[j] = s_goff[r0 + (lane >> 3) + 4 * j];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int r = r0 + (lane >> 3) + 4 * j;
+                            ptx::cp_async_16(sB + r * 128 + ((chunk ^ (r & 7)) << 4),
+                                             off[j] >= 0 ? static_cast<const void*>(base + off[j])
+                                                         : static_cast<const void*>(gsrc),
+                                             off[j] >= 0 ? 16u : 0u);
+                        }
+                    }
+                }
+                ptx::cp_async_mbar_arrive_noinc(&full_bar[stage]);
+                if (++stage == C::kStages) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+        }
+        ptx::cp_async_wait_all();  // nothing still writing into shared memory
     } else {
         // ------------------------------------------------------------ epilogue
         const int quarter = warp & 3;

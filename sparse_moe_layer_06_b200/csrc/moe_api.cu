@@ -428,11 +428,11 @@ int resident_pairs(K kern, int threads, int smem) {
     return n;
 }
 
-template <int EPI, int NMAX, int MB, bool FP8 = false, bool PAIR = false>
+template <int EPI, int NMAX, int MB, bool FP8 = false, bool PAIR = false, int GW = 0>
 int32_t launch_gemm_n(const GemmArgs& a, int grid, cudaStream_t s, const char* name,
                       bool coop = false) {
-    using C = GemmCfg<EPI, NMAX, MB, FP8, PAIR>;
-    auto kern = grouped_gemm_kernel<EPI, NMAX, MB, FP8, PAIR>;
+    using C = GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>;
+    auto kern = grouped_gemm_kernel<EPI, NMAX, MB, FP8, PAIR, GW>;
     int dev = 0;
     cudaGetDevice(&dev);
     static std::atomic<uint64_t> configured{0};
@@ -540,7 +540,19 @@ int32_t launch_gemm(int nmax, int mb, const GemmArgs& a, int64_t max_tiles, cuda
                     const char* name) {
     int grid = static_cast<int>(std::min<int64_t>(sm_count(), std::max<int64_t>(1, max_tiles)));
     if constexpr (EPI == EPI_SWIGLU) {
-        const bool pair = use_pair() && nmax >= 64 && a.gather_tok == nullptr;
+        if (a.gather_tok != nullptr) {
+            // row gather by four dedicated gather warps
+            switch (nmax) {
+                case 16: return launch_gemm_n<EPI, 16, 2, false, false, 4>(a, grid, s, name);
+                case 32: return launch_gemm_n<EPI, 32, 2, false, false, 4>(a, grid, s, name);
+                case 64: return launch_gemm_n<EPI, 64, 2, false, false, 4>(a, grid, s, name);
+                case 128: return launch_gemm_n<EPI, 128, 2, false, false, 4>(a, grid, s, name);
+                case 160: return launch_gemm_n<EPI, 160, 2, false, false, 4>(a, grid, s, name);
+                case 256: return launch_gemm_n<EPI, 256, 2, false, false, 4>(a, grid, s, name);
+                default: return MOE_ERR_UNSUPPORTED;
+            }
+        }
+        const bool pair = use_pair() && nmax >= 64;
         return launch_gemm_mb<EPI, 2>(nmax, a, grid, s, name, pair);
     } else if constexpr (EPI == EPI_LOGITS) {
         if (nmax == 256) {
