@@ -4,7 +4,8 @@ This package is the plain, slow, fp64 reference that the CUDA path is checked
 against.  Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg
 of ``bench.py`` may import it; the product package never does, and the two
 share no code.  All arithmetic lives in ``moe_oracle.c`` (plain C, double
-precision, OpenMP over tokens); this module only builds that file with gcc and
+precision, OpenMP over independent tokens or channels); this module only builds
+that file with gcc and
 marshals arguments through ctypes.
 
 Inputs are torch CPU tensors in the stored dtype (``torch.bfloat16`` or

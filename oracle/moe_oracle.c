@@ -10,7 +10,8 @@
  * (fp64).  Inputs are stored as bf16 or fp32 and are widened exactly to
  * double before use.  Loops run in the plain order of the definitions below;
  * there is no blocking, fusion or reordering beyond what the definitions
- * state.  OpenMP is used only to spread independent tokens over cores.
+ * state.  OpenMP is used only to spread independent tokens (and the
+ * independent channels of the FP8 weight encoder) over cores.
  *
  * What is computed, per token t (x_t is the row x[t, 0:H]):
  *
