@@ -289,6 +289,87 @@ def run_reference(args, cfg, rank, world):
     return 0
 
 
+# ------------------------------------------------------------------ router statistics
+
+def run_router_stats(args, cfg, local, world):
+    """Time moe_router_stats (routing probabilities, selection shares, aux loss,
+    EMA counts) over the workload's T tokens; one rank (an auxiliary line)."""
+    from sparse_moe_layer_06_b200 import moe
+    from sparse_moe_layer_06_b200.workloads import make_router_inputs
+    if world != 1:
+        raise SystemExit("--op router_stats runs on one GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    inp = make_router_inputs(cfg, seed=0, device=dev)
+    p = moe.MoEProblem.from_config(cfg)
+    ws = moe.alloc_workspace(p, moe.MOE_CALL_ROUTER_STATS, device=dev)
+    P = torch.empty(cfg.E, dtype=torch.float32, device=dev)
+    f = torch.empty(cfg.E, dtype=torch.float32, device=dev)
+    aux = torch.empty(1, dtype=torch.float32, device=dev)
+    ema = torch.zeros(cfg.E, dtype=torch.float32, device=dev)
+    ema_total = torch.zeros(1, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        moe.moe_router_stats(p, inp["x"], inp["gate_w"], inp["logit_bias"], P, f, aux, ema,
+                             ema_total, 0.9, ws, stream)
+
+    clocks = ClockSampler(0).start()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    moe.moe_profile_start(args.steps * 8 + 64)
+    torch.cuda.synchronize(dev)
+    launches0 = moe.moe_launch_count()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    ev1.synchronize()
+    wall1 = time.time()
+    launches = moe.moe_launch_count() - launches0
+    kernel_times = moe.moe_profile_stop()
+    clocks.stop()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    status = moe.moe_read_device_status(ws)
+    peaks, peak_kind = read_peaks()
+    hbm_peak = float(peaks["hbm_gbs"])
+    b = 2 if cfg.dtype == torch.bfloat16 else 4
+    bytes_ = cfg.T * cfg.H * b + cfg.E * cfg.H * b + cfg.T * cfg.E * 4
+    flops = 2 * cfg.T * cfg.H * cfg.E
+    dominant = max(kernel_times, key=lambda k: kernel_times[k][1])
+    dom_ms = kernel_times[dominant][1] / max(1, kernel_times[dominant][0])
+    line = {
+        "metric": "router statistics tokens/s (moe_router_stats) on 1 B200",
+        "value": cfg.T / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if cfg.dtype == torch.bfloat16 else "f32",
+        "data": "synthetic (seeded N(0,1) tokens, N(0,0.006) router weights; random init)",
+        "config": {"workload": f"{cfg.name}_router_stats", "T": cfg.T, "H": cfg.H, "E": cfg.E,
+                   "top_k": cfg.top_k,
+                   "l2": (f"x is {cfg.T * cfg.H * b / 1e6:.0f} MB, "
+                          + ("larger than L2 (126 MB): streamed each step" if cfg.T * cfg.H * b > 126e6
+                             else "smaller than L2 (126 MB): not a DRAM-bound measurement"))},
+        "roofline": {"bound": "hbm", "achieved": bytes_ / (ms / 1e3) / 1e9, "peak": hbm_peak,
+                     "unit": "GB/s", "frac": bytes_ / (ms / 1e3) / 1e9 / hbm_peak,
+                     "traffic": None, "kernel": "whole call",
+                     "algorithmic": {"bytes": bytes_, "flops": flops},
+                     "peak_source": peak_kind},
+        "kernels": {k: {"launches": v[0], "ms_per_launch": v[1] / max(1, v[0])}
+                    for k, v in kernel_times.items()},
+        "dominant_kernel_ms": dom_ms,
+        "cpu_baseline": None,
+        "clocks": clocks.summary(wall1 - ms * args.steps / 1e3, wall1),
+        "e2e": None,
+        "gpu_launches": launches,
+        "device_status": status,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 # ------------------------------------------------------------------ our arm
 
 def main():
@@ -306,6 +387,9 @@ def main():
                     help="override T of the workload (smaller cases for profiling)")
     ap.add_argument("--experts", type=int, default=None,
                     help="override E of the workload (smaller cases for profiling)")
+    ap.add_argument("--op", default="forward", choices=["forward", "router_stats"],
+                    help="router_stats: time moe_router_stats (the router's load-balancing "
+                         "statistics) on the workload's tokens instead of the layer")
     ap.add_argument("--weights", default="bf16", choices=["bf16", "fp8"],
                     help="expert weights as stored (fp8: E4M3 codes + power-of-two "
                          "channel scales, moe_forward_fp8)")
@@ -337,6 +421,8 @@ def main():
         return run_reference(args, cfg, rank, world)
 
     from sparse_moe_layer_06_b200 import moe
+    if args.op == "router_stats":
+        return run_router_stats(args, cfg, local, world)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     dist = None

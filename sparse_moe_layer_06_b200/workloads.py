@@ -109,6 +109,16 @@ def make_inputs(cfg: MoEConfig, seed: int = 0, device="cpu") -> dict:
     return dict(x=x, gate_w=gate_w, expert_w=expert_w, shared_w=shared_w, logit_bias=bias)
 
 
+def make_router_inputs(cfg: MoEConfig, seed: int = 0, device="cpu") -> dict:
+    """Only x, gate_w and logit_bias of make_inputs (same draws), without the
+    expert weights."""
+    device = torch.device(device)
+    x = _normal((cfg.T, cfg.H), cfg.x_std, cfg.dtype, device, _gen(device, seed + 0))
+    gate_w = _normal((cfg.E, cfg.H), cfg.w_std, cfg.dtype, device, _gen(device, seed + 1))
+    bias = skew_logit_bias(cfg.E).to(device) if cfg.skew_bias else None
+    return dict(x=x, gate_w=gate_w, logit_bias=bias)
+
+
 def make_x(cfg: MoEConfig, seed: int = 0, device="cpu") -> torch.Tensor:
     """Only the token activations of make_inputs (same draw)."""
     device = torch.device(device)
