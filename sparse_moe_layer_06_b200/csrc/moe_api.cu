@@ -628,6 +628,8 @@ struct RouteOut {
     bool keep_sum;
 };
 
+constexpr int kFusedRouteMaxTokens = 32;  // tokens one CTA routes in the fused launch
+
 // MOE_FUSED_ROUTE=0 keeps the router GEMM and the top-k kernel separate.
 bool fused_route_enabled() {
     static const bool v = env_int("MOE_FUSED_ROUTE", 1) != 0;
@@ -719,8 +721,11 @@ int32_t run_route(const moe_problem* p, const void* x, const void* gate_w, const
                   float* logits, int32_t* count, int32_t* idx, float* w, bool keep_sum,
                   int32_t* status, cudaStream_t s) {
     const LogitsPlan lp = logits_plan(p, true);
+    // fused when every tile has its own SM and each CTA routes at most 32
+    // tokens afterwards (at 128 per CTA the two launches measured faster)
+    const int per_cta = (lp.nmax + lp.splits - 1) / lp.splits;
     if (p->dtype == MOE_BF16 && fused_route_enabled() &&
-        logits_chunks(p) * lp.splits <= sm_count()) {
+        logits_chunks(p) * lp.splits <= sm_count() && per_cta <= kFusedRouteMaxTokens) {
         const RouteOut r{bias, idx, w, count, keep_sum};
         return run_logits_bf16(p, x, gate_w, logits, status, s, lp, &r);
     }
