@@ -469,3 +469,16 @@ def test_fp8_forward_matches_torch_composition():
         for j in range(cfg.top_k):
             ref = ref + r["w"][t, j] * ffn(xq, sx, f64(inp["expert_w"][r["idx"][t, j]]))[0]
         np.testing.assert_allclose(got["out"][t], ref.numpy(), rtol=1e-9, atol=1e-12)
+
+
+def test_router_inputs_are_the_layer_inputs_draws():
+    """make_router_inputs draws exactly the x, gate weight and bias of
+    make_inputs (same seeds), without the expert weights."""
+    import torch
+    from sparse_moe_layer_06_b200.workloads import MoEConfig, make_inputs, make_router_inputs
+    c = MoEConfig("r", T=9, H=64, E=8, top_k=2, I=64, num_shared=1, dtype=torch.bfloat16,
+                  x_std=1.0, w_std=0.02, routed_scale=2.827, clip_limit=10.0, skew_bias=True)
+    full = make_inputs(c, seed=5)
+    r = make_router_inputs(c, seed=5)
+    assert torch.equal(full["x"], r["x"]) and torch.equal(full["gate_w"], r["gate_w"])
+    assert torch.equal(full["logit_bias"], r["logit_bias"])
