@@ -65,34 +65,58 @@ def layer_counts(cfg, idx_cpu, fp8=False):
 
 
 def gate_up_counts(cfg, touched, fp8=False):
-    """Algorithmic FLOPs / bytes of one launch of the grouped gate/up GEMM:
-    gate+up weights of every touched expert (+ shared), the permuted token rows
-    and x (shared expert) read once, h written once (FP8: one byte per
-    element, plus channel and token scales)."""
+    """Algorithmic FLOPs / bytes of one launch of the grouped gate/up GEMM, on
+    the layer roofline's definition: the gate and up weights of every touched
+    expert (+ the shared expert) and the token rows x, each read once (FP8:
+    one byte per weight plus its fp32 row scales).  The permuted token copy and
+    h are implementation traffic and are not credited."""
     T, H, I, k, S = cfg.T, cfg.H, cfg.I, cfg.top_k, cfg.num_shared
     rows = T * (k + S)
     flops = 2 * 2 * rows * H * I
-    e = 1 if fp8 else 2
-    bytes_ = (touched + S) * 2 * I * H * e + rows * H * e + rows * I * e
+    b = 2 if cfg.dtype == torch.bfloat16 else 4
     if fp8:
-        bytes_ += (touched + S) * 2 * I * 4 + T * 4
+        bytes_ = (touched + S) * (2 * I * H + 2 * I * 4) + T * H * b
+    else:
+        bytes_ = (touched + S) * 2 * I * H * b + T * H * b
     return flops, bytes_
 
 
 def down_counts(cfg, touched, scatter_add=False, fp8=False):
-    """One launch of the grouped down GEMM: down weights of every touched expert
-    (+ shared) and h read once; then either the weighted bf16 rows written once
-    (store epilogue) or the fp32 token accumulator read and written once
-    (scatter-add epilogue)."""
+    """One launch of the grouped down GEMM, on the layer roofline's definition:
+    the down weights of every touched expert (+ shared) read once and the
+    layer output written once (FP8: one byte per weight plus its fp32 column
+    scales).  h, the weighted rows and the fp32 accumulator are implementation
+    traffic and are not credited."""
     T, H, I, k, S = cfg.T, cfg.H, cfg.I, cfg.top_k, cfg.num_shared
     rows = T * (k + S)
     flops = 2 * rows * H * I
-    e = 1 if fp8 else 2
-    out_bytes = 2 * T * H * 4 if scatter_add else rows * H * 2
-    bytes_ = (touched + S) * I * H * e + rows * I * e + out_bytes
+    b = 2 if cfg.dtype == torch.bfloat16 else 4
     if fp8:
-        bytes_ += (touched + S) * H * 4
+        bytes_ = (touched + S) * (I * H + H * 4) + T * H * b
+    else:
+        bytes_ = (touched + S) * I * H * b + T * H * b
     return flops, bytes_
+
+
+def kernel_roofline(name, cfg, touched, fp8, ms_per_launch, hbm_peak, tf_peak):
+    """Roofline record of one expert-GEMM launch: algorithmic work on the layer
+    roofline's definition divided by its CUDA-event duration."""
+    if name == "expert_down_combine_gemm":
+        kf, kb = down_counts(cfg, touched, scatter_add=True)
+    elif name in ("expert_down_gemm", "expert_down_gemm_fp8"):
+        kf, kb = down_counts(cfg, touched, fp8=fp8)
+    else:
+        kf, kb = gate_up_counts(cfg, touched, fp8)
+    t = ms_per_launch / 1e3
+    if kb / (hbm_peak * 1e9) >= kf / (tf_peak * 1e12):
+        r = {"bound": "hbm", "achieved": kb / t / 1e9, "peak": hbm_peak, "unit": "GB/s"}
+    else:
+        r = {"bound": "tensor", "achieved": kf / t / 1e12, "peak": tf_peak, "unit": "TFLOP/s"}
+    r["frac"] = r["achieved"] / r["peak"]
+    r["kernel"] = name
+    r["ms_per_launch"] = ms_per_launch
+    r["algorithmic"] = {"bytes": kb, "flops": kf}
+    return r
 
 
 def source_hash():
@@ -121,69 +145,118 @@ def ncu_traffic(kernel: str, workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples every 200 ms; summary() keeps only the
-    samples taken inside a given wall-clock window (the timed region)."""
+    """SM clock, power and clock-event (throttle) reasons of the GPU, sampled
+    during the timed region.  Polls NVML every 10 ms from a thread (so even a
+    timed region of a few tens of milliseconds gets samples); without NVML it
+    falls back to `nvidia-smi -lms 50`.  summary() keeps only the samples
+    taken inside a given wall-clock window.  Nothing here changes a setting."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
     REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    PERIOD_S = 0.010
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, device=None):
         self.gpu = gpu_index
+        self.device = device
         self.proc = None
-        self.samples = []  # (wall time, fields)
+        self.samples = []  # (wall time, sm MHz, sm max MHz, power W, [reason names])
         self.thread = None
+        self.stop_flag = threading.Event()
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        if self.device is not None:
+            uuid = str(torch.cuda.get_device_properties(self.device).uuid)
+            for cand in (uuid, "GPU-" + uuid):
+                try:
+                    return pynvml, pynvml.nvmlDeviceGetHandleByUUID(cand)
+                except pynvml.NVMLError:
+                    pass
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
-            return self
-        self.thread = threading.Thread(target=self._read, daemon=True)
+            nv, h = self._nvml_handle()
+            bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+            smax = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        except Exception:  # no NVML binding or device: use nvidia-smi
+            return self._start_smi()
+        self.source = "nvml, 10 ms"
+
+        def poll():
+            while not self.stop_flag.is_set():
+                try:
+                    sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                    pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((time.time(), sm, smax, pw,
+                                         [k for k, b in bits.items() if r & b]))
+                except Exception:
+                    pass
+                self.stop_flag.wait(self.PERIOD_S)
+        self.thread = threading.Thread(target=poll, daemon=True)
         self.thread.start()
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
-                self.samples.append((time.time(), parts))
-
-    def stop(self):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-            if self.thread:
-                self.thread.join(timeout=2)
-
-    def summary(self, t0: float, t1: float):
-        rows = [r for (t, r) in self.samples if t0 <= t <= t1]
-        mine = [r for r in rows if r[0] == str(self.gpu)] or rows
-        if not mine:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples in window"],
-                    "samples": 0}
+    def _start_smi(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return self
+        self.source = "nvidia-smi, 50 ms"
 
         def num(x):
             try:
                 return float(x)
             except ValueError:
                 return None
-        sm = [num(r[1]) for r in mine if num(r[1]) is not None]
-        smax = [num(r[2]) for r in mine if num(r[2]) is not None]
-        pw = [num(r[3]) for r in mine if num(r[3]) is not None]
-        reasons = sorted({self.REASONS[i] for r in mine for i in range(4)
-                          if r[5 + i].lower() in ("active", "1")})
+
+        def read():
+            for line in self.proc.stdout:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[0] == str(self.gpu):
+                    reasons = [self.REASONS[i] for i in range(4)
+                               if parts[5 + i].lower() in ("active", "1")]
+                    self.samples.append((time.time(), num(parts[1]), num(parts[2]),
+                                         num(parts[3]), reasons))
+        self.thread = threading.Thread(target=read, daemon=True)
+        self.thread.start()
+        return self
+
+    def stop(self):
+        self.stop_flag.set()
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+
+    def summary(self, t0: float, t1: float):
+        mine = [r for r in self.samples if t0 <= r[0] <= t1]
+        if not mine:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples in window"],
+                    "samples": 0, "source": self.source}
+        sm = [r[1] for r in mine if r[1] is not None]
+        smax = [r[2] for r in mine if r[2] is not None]
+        pw = [r[3] for r in mine if r[3] is not None]
+        reasons = sorted({x for r in mine for x in r[4]})
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
                 "power_w_max": max(pw) if pw else None,
-                "reasons": reasons, "samples": len(mine)}
+                "reasons": reasons, "samples": len(mine), "source": self.source}
 
 
 # ------------------------------------------------------------------ ranks
@@ -314,7 +387,7 @@ def run_router_stats(args, cfg, local, world):
         moe.moe_router_stats(p, inp["x"], inp["gate_w"], inp["logit_bias"], P, f, aux, ema,
                              ema_total, 0.9, ws, stream)
 
-    clocks = ClockSampler(0).start()
+    clocks = ClockSampler(0, dev).start()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -372,6 +445,78 @@ def run_router_stats(args, cfg, local, world):
 
 # ------------------------------------------------------------------ our arm
 
+def time_steps(step, n, stream, dist=None, device=None):
+    """Device time of n back-to-back steps (CUDA events on the launching
+    stream, synchronised on both sides, max over ranks), in ms per step."""
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(n):
+        step()
+    ev1.record(stream)
+    ev1.synchronize()
+    return max_over_ranks(ev0.elapsed_time(ev1), dist, device) / n
+
+
+def kernel_times(moe, step, n, device=None):
+    """Per-kernel CUDA-event durations over n steps (the library records an
+    event pair around each launch on its stream).  Those events also keep
+    consecutive launches from overlapping, so this runs as its own pass after
+    the timed region; returns {name: (launches, total ms)}."""
+    torch.cuda.synchronize(device)
+    moe.moe_profile_start(n * 16 + 64)
+    for _ in range(n):
+        step()
+    torch.cuda.synchronize(device)
+    return moe.moe_profile_stop()
+
+
+def measure_workload(moe, cfg, inp, x, dev, stream, steps, warmup, fp8_weights=None):
+    """Time one workload on weights already resident (a sub-record of the bench
+    line): ms/step, tokens/s, layer roofline fraction and the dominant
+    kernel's roofline record."""
+    p = moe.MoEProblem.from_config(cfg)
+    ws = moe.alloc_workspace(p, moe.MOE_CALL_FORWARD, device=dev)
+    out = torch.empty(cfg.T, cfg.H, dtype=cfg.dtype, device=dev)
+    idx = torch.empty(cfg.T, cfg.top_k, dtype=torch.int32, device=dev)
+    w = torch.empty(cfg.T, cfg.top_k, dtype=torch.float32, device=dev)
+    bias = inp["logit_bias"]
+
+    def step():
+        moe.moe_forward(p, x, inp["gate_w"], bias, inp["expert_w"], inp["shared_w"], out, idx, w,
+                        ws, stream)
+    for _ in range(warmup):
+        step()
+    ms = time_steps(step, steps, stream, None, dev)
+    kt = kernel_times(moe, step, steps, dev)
+    status = moe.moe_read_device_status(ws)
+    peaks, _ = read_peaks()
+    hbm_peak = float(peaks["hbm_gbs"])
+    tf_peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    idx_cpu = idx.cpu()
+    flops, bytes_, touched = layer_counts(cfg, idx_cpu)
+    t_s = ms / 1e3
+    roof_t = max(flops / (tf_peak * 1e12), bytes_ / (hbm_peak * 1e9))
+    dom = max(kt, key=lambda k: kt[k][1])
+    rec = {"workload": cfg.name, "T": cfg.T, "ms_per_step": ms, "tokens_per_s": cfg.T / t_s,
+           "tflops": flops / t_s / 1e12, "layer_roofline_frac": roof_t / t_s,
+           "layer_bound": "tensor" if flops / (tf_peak * 1e12) > bytes_ / (hbm_peak * 1e9)
+           else "hbm",
+           "touched_experts": touched,
+           "dominant": kernel_roofline(dom, cfg, touched, False, kt[dom][1] / max(1, kt[dom][0]),
+                                       hbm_peak, tf_peak),
+           "kernels": {k: v[1] / max(1, v[0]) for k, v in kt.items()},
+           "device_status": status}
+    counts = torch.bincount(idx_cpu.reshape(-1).long(), minlength=cfg.E).float()
+    rec["max_expert_share"] = float(counts.max() / cfg.T)
+    del ws, out, idx, w
+    torch.cuda.empty_cache()
+    return rec
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -380,6 +525,8 @@ def main():
     ap.add_argument("--config", default="hy4_prefill", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the decode / skewed sub-records of a Hy4 line")
     ap.add_argument("--e2e-steps", type=int, default=None,
                     help="steps of the end-to-end measurement (default: --steps, so that "
                          "both run equally long under the power cap)")
@@ -403,6 +550,7 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     cfg = CONFIGS[args.config]
+    base_cfg = cfg
     if args.tokens is not None or args.experts is not None:
         from dataclasses import replace
         cfg = replace(cfg, T=args.tokens or cfg.T, E=args.experts or cfg.E,
@@ -473,7 +621,7 @@ def main():
         forward(inp["x"], out, stream)
 
     gpu_index = local if torch.cuda.device_count() > 1 else 0
-    clocks = ClockSampler(gpu_index).start()
+    clocks = ClockSampler(gpu_index, dev).start()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -481,28 +629,18 @@ def main():
         raise RuntimeError("device error word set during warm-up")
 
     # ---------------- timed region (device time, CUDA events, max over ranks)
-    moe.moe_profile_start(args.steps * 16 + 64)
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
     launches0 = moe.moe_launch_count()
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
-    for _ in range(args.steps):
-        step()
-    ev1.record(stream)
-    wall0 = time.time()
-    ev1.synchronize()
+    ms_per_step = time_steps(step, args.steps, stream, dist, dev)
     wall1 = time.time()
     launches = moe.moe_launch_count() - launches0
+    clock_rec = clocks.summary(wall1 - ms_per_step * args.steps / 1e3, wall1)
+    # per-kernel durations: the same number of steps again, with an event pair
+    # around every launch (a separate pass: the events keep launches apart)
+    kt = kernel_times(moe, step, args.steps, dev)
     if dist:
         dist.barrier()
-    kernel_times = moe.moe_profile_stop()
-    clocks.stop()
-    ms = max_over_ranks(ev0.elapsed_time(ev1), dist, dev)
     status = moe.moe_read_device_status(ws)
-    ms_per_step = ms / args.steps
+    ms = ms_per_step * args.steps
 
     # ---------------- end to end: host buffers, copies inside the timed region.
     # Each step copies its tokens in from pinned host memory, runs the layer
@@ -553,10 +691,32 @@ def main():
     if dist:
         dist.barrier()
 
+    # ---------------- the other Hy4-shape workloads on the same weights
+    # (decode: HBM-bound weight stream; skewed routing: tensor-bound), timed
+    # the same way after the headline measurement, single GPU only
+    workloads = None
+    hy4 = ("hy4_prefill", "hy4_decode", "hy4_skew")
+    if (world == 1 and not fp8 and not args.no_workloads and base_cfg.name in hy4
+            and args.tokens is None and args.experts is None):
+        workloads = {}
+        from sparse_moe_layer_06_b200.workloads import skew_logit_bias
+        for name in hy4:
+            if name == base_cfg.name:
+                continue
+            c = CONFIGS[name]
+            winp = dict(inp)
+            winp["logit_bias"] = skew_logit_bias(c.E).to(dev) if c.skew_bias else None
+            xw = make_x(c, seed=rank_token_seed(rank), device=dev)
+            workloads[name] = measure_workload(moe, c, winp, xw, dev, stream, args.steps,
+                                               args.warmup)
+            del xw
+
     if rank != 0:
+        clocks.stop()
         if dist:
             dist.destroy_process_group()
         return 0
+    clocks.stop()
 
     # ---------------- derived numbers
     peaks, peak_kind = read_peaks()
@@ -573,28 +733,14 @@ def main():
     roof_t_nominal = max(flops / 2250e12, bytes_ / 8000e9)
 
     per_kernel = {k: {"launches": v[0], "ms_per_launch": v[1] / max(1, v[0]),
-                      "share": v[1] / max(1e-9, sum(x[1] for x in kernel_times.values()))}
-                  for k, v in kernel_times.items()}
-    dominant = max(kernel_times, key=lambda k: kernel_times[k][1])
-    dom_ms = kernel_times[dominant][1] / max(1, kernel_times[dominant][0])
-    if dominant == "expert_down_combine_gemm":
-        kf, kb = down_counts(cfg, touched, scatter_add=True)
-    elif dominant in ("expert_down_gemm", "expert_down_gemm_fp8"):
-        kf, kb = down_counts(cfg, touched, fp8=fp8)
-    else:
-        kf, kb = gate_up_counts(cfg, touched, fp8)
-    dom_s = dom_ms / 1e3
-    t_hbm = kb / (hbm_peak * 1e9)
-    t_tc = kf / (tf_peak * 1e12)
-    if t_hbm >= t_tc:
-        roof = {"bound": "hbm", "achieved": kb / dom_s / 1e9, "peak": hbm_peak, "unit": "GB/s"}
-    else:
-        roof = {"bound": "tensor", "achieved": kf / dom_s / 1e12, "peak": tf_peak,
-                "unit": "TFLOP/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
+                      "share": v[1] / max(1e-9, sum(x[1] for x in kt.values()))}
+                  for k, v in kt.items()}
+    dominant = max(kt, key=lambda k: kt[k][1])
+    dom_ms = kt[dominant][1] / max(1, kt[dominant][0])
+    roof = kernel_roofline(dominant, cfg, touched, fp8, dom_ms, hbm_peak, tf_peak)
     roof["traffic"] = ncu_traffic(dominant, cfg.name)
-    roof["kernel"] = dominant
-    roof["algorithmic"] = {"bytes": kb, "flops": kf}
+    roof["timing"] = ("CUDA events around each launch on its stream, over a pass of "
+                      f"{args.steps} steps right after the timed region")
     roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" \
         else "fallback"
     if fp8 and roof["bound"] == "tensor":
@@ -637,8 +783,9 @@ def main():
                            "touched_experts": touched, "peak_source": peak_kind},
         "roofline": roof,
         "kernels": per_kernel,
+        "workloads": workloads,
         "cpu_baseline": cpu_base,
-        "clocks": clocks.summary(wall1 - ms / 1e3, wall1),
+        "clocks": clock_rec,
         "e2e": {"value": whole_job_rate(cfg.T * args.e2e_steps, world, e2e_ms / 1e3),
                 "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

@@ -95,6 +95,18 @@ size_t moe_workspace_size(const moe_problem* problem, int32_t call);
 const char* moe_status_string(int32_t status);
 
 /*
+ * moe_expert_tile_rows -- the token-row tile widths moe_forward and
+ * moe_forward_fp8 use for this problem (host only, no CUDA call): each
+ * expert's rows (and the shared expert's T rows) are cut into
+ * c = ceil(rows / width) chunks of ceil16(ceil(rows / c)) rows, the last one
+ * shorter, and every chunk is one token tile of the gate/up (*gate_up_rows)
+ * or the down GEMM (*down_rows).  Useful to test or profile every tile of a
+ * schedule.  Both outputs are host pointers.
+ */
+int32_t moe_expert_tile_rows(const moe_problem* problem, int32_t* gate_up_rows,
+                             int32_t* down_rows);
+
+/*
  * moe_router_logits -- the router's gate GEMM:
  *   logits[t, e] = sum_h x[t, h] * gate_w[e, h]      (fp32 [T, E], device, out)
  * x: [T, H] device; gate_w: [E, H] device (nn.Linear weight layout).
@@ -174,10 +186,15 @@ int32_t moe_combine(const moe_problem* problem, const void* y_perm, const int32_
 /*
  * moe_forward -- the whole layer in one call: route, dispatch, grouped
  * gate/up GEMM with the clamp + SwiGLU fused into its epilogue, grouped down
- * GEMM whose epilogue multiplies by the routing weight and scatter-adds into
- * an fp32 token accumulator (the shared expert is one more group with weight
- * 1), then a cast to the output dtype.  The fp32 scatter-add makes the output
- * bits depend on the order of atomic additions (within the stated tolerance).
+ * GEMM whose epilogue multiplies each row by its routing weight (the shared
+ * expert is one more group, with weight 1) and stores the weighted rows, then
+ * a combine kernel that adds each token's top_k rows and its shared-expert
+ * row in slot order, in fp32, and writes the output dtype.  Every sum is
+ * taken in a fixed order, so the output is bitwise reproducible from run to
+ * run.  (Setting MOE_COMBINE=atomic in the environment selects the other
+ * form: the down epilogue scatter-adds into an fp32 token accumulator, whose
+ * result bits then depend on the order of the atomic additions, within the
+ * stated tolerance.)
  *   x            [T, H] device
  *   gate_w       [E, H] device
  *   logit_bias   [E] fp32 device or NULL
@@ -208,8 +225,11 @@ int32_t moe_forward(const moe_problem* problem, const void* x, const void* gate_
  *    (e.g. T <= 1023 tokens at E = 256); larger problems return
  *    MOE_ERR_WORKSPACE and enqueue nothing.
  *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *    (cudaGetSymbolAddress) with that device current, and keeps it for the
+ *    life of the process; make that first call before any stream capture.
+ *    A device reset (cudaDeviceReset, or anything else that destroys the
+ *    primary context) invalidates the kept address: do not call this entry
+ *    point again in a process that has reset the device.
  *  - All calls share the one array and it keeps the last call's contents:
  *    calls that overlap on the GPU (different streams, or different host
  *    threads, on one device) race and corrupt each other's logits.  Order

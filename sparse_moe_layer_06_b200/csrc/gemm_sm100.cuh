@@ -154,6 +154,24 @@ struct GemmArgs {
     float h_scale;      // a power of two
     float h_scale_inv;  // its exact reciprocal
     int32_t* status;           // device error word
+    // K order: 0 = every tile runs K from its first step; 1 = each tile starts
+    // at a tile-dependent step and wraps around (the sum order of a tile is
+    // still fixed), so CTAs running together read different K bands of the
+    // weights instead of the same one in lockstep
+    int32_t k_rotate;
+    // Programmatic dependent launch.  Before waiting for the grid it depends
+    // on, the producer pulls the first prefetch_ksteps weight steps of this
+    // CTA's first tile into L2 (weights never depend on an earlier launch);
+    // every thread that reads an earlier launch's output waits first.  With
+    // pdl_trigger_early the next launch may start as soon as this grid has
+    // passed that wait (otherwise when each CTA finishes its tiles).
+    int32_t prefetch_ksteps;
+    int32_t pdl_trigger_early;
+    // Weight read-ahead: with each stage's copies the producer also pulls the
+    // weight box pf_dist steps further along the tile into L2, so more weight
+    // bytes are on their way from DRAM than the shared-memory ring holds
+    // (0 = off)
+    int32_t pf_dist;
 };
 
 // Compile-time shape of one instantiation.
@@ -258,6 +276,15 @@ __device__ __forceinline__ bool decode_tile(int t, int nblk, int nseg, const Sme
     return n > 0;
 }
 
+// First K step (relative to the tile's range of `span` steps) of a tile whose
+// K loop is rotated: spread over the range by weight block, shifted by
+// segment and chunk, so that concurrently running tiles (consecutive weight
+// blocks of a few segments) start at different K offsets.
+__device__ __forceinline__ int k_rotation(const TileInfo& ti, int span, int nblk) {
+    if (span <= 1) return 0;
+    return (ti.blk * span / nblk + ti.seg * 7 + ti.chunk * 3) % span;
+}
+
 // Reciprocal of d >= 1 with the hardware approximation (relative error ~2^-23;
 // 1/inf = 0, the correct limit of the SiLU gate).
 __device__ __forceinline__ float fast_rcp(float d) {
@@ -312,7 +339,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
     ss.chunk_len = s_sched + 4 * (nseg + 1);
     if (args.sched) {
         for (int i = threadIdx.x; i < 5 * (nseg + 1); i += blockDim.x)
-            s_sched[i] = __ldg(args.sched + i);
+            s_sched[i] = __ldcg(args.sched + i);  // (L2: written by an earlier launch)
     } else if (threadIdx.x == 0) {
         const int cl = args.single_chunk_len;
         ss.prefix[0] = 0;
@@ -368,6 +395,18 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
     const int total_tiles = ss.prefix[nseg] * nblk * ksplit;
     const int ksteps = args.K / C::kKStep;
 
+    // K rotation of a tile (PAIR: of the pair's shared tile, so that both CTAs
+    // fill every stage with the same K step)
+    auto k_rot = [&](const TileInfo& ti, int span) -> int {
+        if (!args.k_rotate) return 0;
+        if constexpr (PAIR) {
+            TileInfo tp = ti;
+            tp.blk = ti.blk >> 1;
+            return k_rotation(tp, span, nblk);
+        } else {
+            return k_rotation(ti, span, nblk_cta);
+        }
+    };
     auto fail = [&](int code) {
         *abort_flag = 1;
         set_device_error(args.status, code);
@@ -397,6 +436,35 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
         // token chunk of that segment: keep them in L2 rather than streaming
         const uint64_t pol_ws = pol_x;
         const bf16_raw_ptr gsrc = reinterpret_cast<bf16_raw_ptr>(args.gather_src);
+        if (C::kSwiGLU || C::kDown) {
+            // weights of this CTA's first tile into L2 while the launch this
+            // one depends on may still be running (weights are never written)
+            if (lane == 0 && args.prefetch_ksteps > 0) {
+                for (int t = unit; t < total_tiles; t += units) {
+                    TileInfo ti;
+                    if (!decode(t, ti)) continue;
+                    const CUtensorMap* tA = ti.special ? &args.tmA1 : &args.tmA0;
+                    const int a_base = ti.special ? 0 : ti.seg * args.a_seg_stride;
+                    const uint64_t pw = ti.special ? pol_ws : pol_w;
+                    const int rot = k_rot(ti, ksteps);
+                    const int n = args.prefetch_ksteps < ksteps ? args.prefetch_ksteps : ksteps;
+                    for (int i = 0; i < n; ++i) {
+                        const int kb = i + rot < ksteps ? i + rot : i + rot - ksteps;
+                        const int k0 = kb * C::kKStep;
+                        if constexpr (C::kDown)
+                            ptx::tma_prefetch_3d(tA, 0, a_base + args.a_off0 + k0,
+                                                 ti.blk * (FP8 ? MB : 2 * MB), pw);
+                        else
+                            ptx::tma_prefetch_3d(tA, k0, ti.blk * 128, a_base + args.a_off0, pw);
+                    }
+                    break;
+                }
+            }
+        }
+        // token rows (and, for a gathered tile, their indices) come from
+        // earlier launches
+        ptx::grid_dep_wait();
+        if (args.pdl_trigger_early) ptx::grid_dep_launch();
         uint32_t stage = 0, phase = 0;
         uint32_t armed = 0, armed_phase = 0;  // per-stage bits (lane 0)
         bool ok = true;
@@ -405,6 +473,8 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
             const int ks = t % ksplit;
             if (!decode(t, ti)) continue;
             const int kb_begin = ks * ksteps / ksplit, kb_end = (ks + 1) * ksteps / ksplit;
+            const int span = kb_end - kb_begin;
+            const int rot = k_rot(ti, span);
             const CUtensorMap* tA = ti.special ? &args.tmA1 : &args.tmA0;
             const CUtensorMap* tB = ti.special ? args.tmB1 : args.tmB0;
             const int a_base = ti.special ? 0 : ti.seg * args.a_seg_stride;
@@ -431,7 +501,8 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
             const uint32_t bytes =
                 PAIR ? 2u * (C::kABytes + b_rows * 128) : C::kABytes + (gather ? 0 : ti.n_mma * 128);
             // (gathered rows arrive through cp.async, counted as arrivals)
-            for (int kb = kb_begin; kb < kb_end; ++kb) {
+            for (int i = 0; i < span; ++i) {
+                const int kb = kb_begin + (i + rot < span ? i + rot : i + rot - span);
                 int got = 1;
                 if (lane == 0) got = ptx::mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag);
                 got = __shfl_sync(0xffffffffu, got, 0);
@@ -510,6 +581,17 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
                             }
                         }
                     }
+                    if ((C::kSwiGLU || C::kDown) && args.pf_dist > 0 && i + args.pf_dist < span) {
+                        // read-ahead of a later weight box of this tile into L2
+                        const int ia = i + args.pf_dist;
+                        const int kp = kb_begin + (ia + rot < span ? ia + rot : ia + rot - span);
+                        const int kp0 = kp * C::kKStep;
+                        if constexpr (C::kDown)
+                            ptx::tma_prefetch_3d(tA, 0, a_base + args.a_off0 + kp0,
+                                                 ti.blk * (FP8 ? MB : 2 * MB), pw);
+                        else
+                            ptx::tma_prefetch_3d(tA, kp0, ti.blk * 128, a_base + args.a_off0, pw);
+                    }
                 }
                 if (++stage == C::kStages) {
                     stage = 0;
@@ -517,6 +599,8 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
                 }
             }
         }
+        // every copy of this CTA is issued: the next launch may start
+        if (!args.pdl_trigger_early) ptx::grid_dep_launch();
         // never leave with copies still writing into this CTA's shared memory
         ptx::cp_async_wait_all();
         __syncwarp();
@@ -554,7 +638,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
                 TileInfo ti;
                 const int ks = t % ksplit;
                 if (!decode(t, ti)) continue;
-                const int kb_begin = ks * ksteps / ksplit, kb_end = (ks + 1) * ksteps / ksplit;
+                const int span = (ks + 1) * ksteps / ksplit - ks * ksteps / ksplit;
                 if (!ptx::mbar_wait(&acce_bar[acc], acc_phase ^ 1, abort_flag)) {
                     fail(DEV_ERR_TIMEOUT);
                     break;
@@ -563,7 +647,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
                 const uint32_t d0 = tmem_base + acc * C::kAccCols;
                 const uint32_t idesc = FP8 ? ptx::idesc_e4m3_f32(kM, ti.n_mma, kAMajor, 0)
                                            : ptx::idesc_bf16_f32(kM, ti.n_mma, kAMajor, 0);
-                for (int kb = kb_begin; kb < kb_end; ++kb) {
+                for (int i = 0; i < span; ++i) {
                     if (!ptx::mbar_wait(&full_bar[stage], phase, abort_flag)) {
                         fail(DEV_ERR_TIMEOUT);
                         ok = false;
@@ -577,7 +661,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
                     const uint32_t b_addr = a_addr + C::kABytes;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
-                        const uint32_t accum = (kb > kb_begin || kk > 0) ? 1u : 0u;
+                        const uint32_t accum = (i > 0 || kk > 0) ? 1u : 0u;
                         const uint64_t bdesc = ptx::smem_desc_sw128(b_addr + kk * 32, 16, 1024);
 #pragma unroll
                         for (int j = 0; j < MB; ++j) {
@@ -617,6 +701,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
         // copies have landed (at once for tiles it has no rows of)
         const int gw = warp - 2 - C::kEpiWarps;
         const bf16_raw_ptr gsrc = reinterpret_cast<bf16_raw_ptr>(args.gather_src);
+        ptx::grid_dep_wait();  // the row indices come from an earlier launch
         uint32_t stage = 0, phase = 0;
         bool ok = true;
         for (int t = unit; ok && t < total_tiles; t += units) {
@@ -624,6 +709,8 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
             const int ks = t % ksplit;
             if (!decode(t, ti)) continue;
             const int kb_begin = ks * ksteps / ksplit, kb_end = (ks + 1) * ksteps / ksplit;
+            const int span = kb_end - kb_begin;
+            const int rot = k_rot(ti, span);
             const bool gather = args.gather_tok != nullptr && !ti.special;
             const int ngroups = ti.n_mma >> 4;
             if (gather) {
@@ -641,7 +728,8 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
                 }
                 __syncwarp();
             }
-            for (int kb = kb_begin; kb < kb_end; ++kb) {
+            for (int i = 0; i < span; ++i) {
+                const int kb = kb_begin + (i + rot < span ? i + rot : i + rot - span);
                 int got = 1;
                 if (lane == 0) got = ptx::mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag);
                 got = __shfl_sync(0xffffffffu, got, 0);
@@ -681,6 +769,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
         const int quarter = warp & 3;
         const int half = (warp - 2) >> 2;  // which of the two warps on this quarter
         const int row_in_tile = quarter * 32 + lane;
+        ptx::grid_dep_wait();  // row metadata and outputs are shared with earlier launches
         uint32_t acc = 0, acc_phase = 0;
         uint32_t mi = 0, meta_phase = 0;
         for (int t = unit; t < total_tiles; t += units) {
@@ -839,6 +928,10 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
                         ptx::reg_fence(v);
                         if constexpr (EPI == EPI_DOWN_ATOMIC) {
                             float* oacc = reinterpret_cast<float*>(args.out);
+                            // each accumulator element takes top_k + 1 additions spread
+                            // over the whole launch: keep its lines in L2 between them
+                            const uint64_t pol_acc = args.l2_hints ? ptx::policy_evict_last()
+                                                                   : ptx::policy_evict_normal();
 #pragma unroll
                             for (int j = 0; j < 16; ++j) {
                                 const int c = c0 + j;
@@ -846,8 +939,9 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
                                     const int tok = w_tok[c];
                                     if (static_cast<unsigned>(tok) <
                                         static_cast<unsigned>(args.n_tokens)) {
-                                        atomicAdd(oacc + static_cast<size_t>(tok) * args.out_ld + m,
-                                                  w_wt[c] * v[j]);
+                                        ptx::red_add_f32(
+                                            oacc + static_cast<size_t>(tok) * args.out_ld + m,
+                                            w_wt[c] * v[j], pol_acc);
                                     } else {
                                         set_device_error(args.status, DEV_ERR_BAD_INDEX);
                                     }

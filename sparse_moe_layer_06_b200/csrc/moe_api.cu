@@ -11,6 +11,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "../../include/moe.h"
@@ -110,6 +111,22 @@ struct ElemType {
 constexpr ElemType kBF16{CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2};
 constexpr ElemType kU8{CU_TENSOR_MAP_DATA_TYPE_UINT8, 1};
 
+int env_int(const char* name, int dflt);
+
+// L2 sector promotion of the expert-weight tensor maps (MOE_L2_PROMO: 0 none,
+// 1 64 B, 2 128 B, 3 256 B; default 256 B).  A weight tile row is 128 bytes
+// per pipeline stage; with 256-byte promotion the next stage's 128 bytes of
+// the same row come in with it.
+CUtensorMapL2promotion weight_l2_promotion() {
+    const int v = env_int("MOE_L2_PROMO", 3);
+    switch (v) {
+        case 0: return CU_TENSOR_MAP_L2_PROMOTION_NONE;
+        case 1: return CU_TENSOR_MAP_L2_PROMOTION_L2_64B;
+        case 2: return CU_TENSOR_MAP_L2_PROMOTION_L2_128B;
+        default: return CU_TENSOR_MAP_L2_PROMOTION_L2_256B;
+    }
+}
+
 // 2D row-major [rows, cols] tensor, box = one 128-byte row segment x box_rows
 // rows, 128-byte swizzle, zero fill outside the tensor.
 bool make_tmap(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int box_rows,
@@ -141,7 +158,7 @@ bool make_tmap_gateup(CUtensorMap* m, const void* ptr, int64_t n_mats, int64_t I
     cuuint32_t estr[3] = {1u, 1u, 1u};
     CUresult r = fn(m, et.dt, 3, const_cast<void*>(ptr), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                    weight_l2_promotion(), CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -163,7 +180,7 @@ bool make_tmap_down(CUtensorMap* m, const void* ptr, int64_t rows, int64_t H, in
     cuuint32_t estr[3] = {1u, 1u, 1u};
     CUresult r = fn(m, et.dt, 3, const_cast<void*>(ptr), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                    weight_l2_promotion(), CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -216,7 +233,7 @@ bool nmax_supported(int n) {
 // for a 4-deep pipeline of gate+up weight tiles; larger segments get 256.
 // MOE_NMAX in the environment overrides it (tuning knob).
 int pick_nmax(double mean_rows) {
-    static const int forced = [] {
+    const int forced = [] {
         const int v = env_int("MOE_NMAX", 0);
         return nmax_supported(v) ? v : 0;
     }();
@@ -233,7 +250,7 @@ int pick_nmax(double mean_rows) {
 // re-read the weights more often, which costs power under the 1 kW cap more
 // than the double-buffered accumulator gains).  MOE_DOWN_NMAX overrides.
 int pick_down_nmax(int nmax_gu) {
-    static const int forced = [] {
+    const int forced = [] {
         const int v = env_int("MOE_DOWN_NMAX", 0);
         return nmax_supported(v) ? v : 0;
     }();
@@ -246,7 +263,7 @@ int pick_down_nmax(int nmax_gu) {
 // the token-tile re-reads (the down GEMM is bound by the bulk-copy rows it
 // issues).  MOE_DOWN_MB overrides.
 int pick_down_mb(int nmax) {
-    static const int forced = [] {
+    const int forced = [] {
         const int v = env_int("MOE_DOWN_MB", 0);
         return (v == 1 || v == 2) ? v : 0;
     }();
@@ -404,6 +421,26 @@ T* at(void* ws, size_t off) {
 
 // ------------------------------------------------------------------ GEMM launch
 
+// Kernel launch on stream s; with pdl the launch may begin before the
+// previous launch on the stream has finished (programmatic stream
+// serialization): the kernel must then wait (griddepcontrol.wait) before it
+// reads anything the previous launch writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kern)(KArgs...), int grid, int threads, int smem, cudaStream_t s,
+                      bool pdl, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(static_cast<unsigned>(threads));
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // Clusters of two CTAs (one per SM) of `kern` that can be resident at once.
 template <typename K>
 int resident_pairs(K kern, int threads, int smem) {
@@ -430,7 +467,7 @@ int resident_pairs(K kern, int threads, int smem) {
 
 template <int EPI, int NMAX, int MB, bool FP8 = false, bool PAIR = false, int GW = 0>
 int32_t launch_gemm_n(const GemmArgs& a, int grid, cudaStream_t s, const char* name,
-                      bool coop = false) {
+                      bool coop = false, bool pdl = false) {
     using C = GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>;
     auto kern = grouped_gemm_kernel<EPI, NMAX, MB, FP8, PAIR, GW>;
     int dev = 0;
@@ -460,13 +497,15 @@ int32_t launch_gemm_n(const GemmArgs& a, int grid, cudaStream_t s, const char* n
         cfg.blockDim = dim3(C::kThreads);
         cfg.dynamicSmemBytes = C::kSmemBytes;
         cfg.stream = s;
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 2;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = pdl ? 2 : 1;
         MOE_LAUNCH(name, s, if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return MOE_ERR_CUDA);
     } else if (coop) {
         // every CTA resident at once (the fused routing phase waits across CTAs)
@@ -482,7 +521,8 @@ int32_t launch_gemm_n(const GemmArgs& a, int grid, cudaStream_t s, const char* n
         cfg.numAttrs = 1;
         MOE_LAUNCH(name, s, if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return MOE_ERR_CUDA);
     } else {
-        MOE_LAUNCH(name, s, kern<<<grid, C::kThreads, C::kSmemBytes, s>>>(a));
+        MOE_LAUNCH(name, s, if (launch_ex(kern, grid, C::kThreads, C::kSmemBytes, s, pdl, a) !=
+                                cudaSuccess) return MOE_ERR_CUDA);
     }
     return MOE_OK;
 }
@@ -493,28 +533,28 @@ int32_t launch_gemm_n(const GemmArgs& a, int grid, cudaStream_t s, const char* n
 // measured slower at the Hy4 prefill shapes (the two CTAs advance in
 // lockstep), and only about 1% faster on the tensor-bound skewed batch.
 bool use_pair() {
-    static const bool v = env_int("MOE_PAIR", 0) != 0;
+    const bool v = env_int("MOE_PAIR", 0) != 0;
     return v;
 }
 
 template <int EPI, int MB, bool FP8 = false>
 int32_t launch_gemm_mb(int nmax, const GemmArgs& a, int grid, cudaStream_t s, const char* name,
-                       bool pair = false) {
+                       bool pair = false, bool pdl = false) {
     switch (nmax) {
-        case 16: return launch_gemm_n<EPI, 16, MB, FP8>(a, grid, s, name);
-        case 32: return launch_gemm_n<EPI, 32, MB, FP8>(a, grid, s, name);
+        case 16: return launch_gemm_n<EPI, 16, MB, FP8>(a, grid, s, name, false, pdl);
+        case 32: return launch_gemm_n<EPI, 32, MB, FP8>(a, grid, s, name, false, pdl);
         case 64:
-            return pair ? launch_gemm_n<EPI, 64, MB, FP8, true>(a, grid, s, name)
-                        : launch_gemm_n<EPI, 64, MB, FP8>(a, grid, s, name);
+            return pair ? launch_gemm_n<EPI, 64, MB, FP8, true>(a, grid, s, name, false, pdl)
+                        : launch_gemm_n<EPI, 64, MB, FP8>(a, grid, s, name, false, pdl);
         case 128:
-            return pair ? launch_gemm_n<EPI, 128, MB, FP8, true>(a, grid, s, name)
-                        : launch_gemm_n<EPI, 128, MB, FP8>(a, grid, s, name);
+            return pair ? launch_gemm_n<EPI, 128, MB, FP8, true>(a, grid, s, name, false, pdl)
+                        : launch_gemm_n<EPI, 128, MB, FP8>(a, grid, s, name, false, pdl);
         case 160:
-            return pair ? launch_gemm_n<EPI, 160, MB, FP8, true>(a, grid, s, name)
-                        : launch_gemm_n<EPI, 160, MB, FP8>(a, grid, s, name);
+            return pair ? launch_gemm_n<EPI, 160, MB, FP8, true>(a, grid, s, name, false, pdl)
+                        : launch_gemm_n<EPI, 160, MB, FP8>(a, grid, s, name, false, pdl);
         case 256:
-            return pair ? launch_gemm_n<EPI, 256, MB, FP8, true>(a, grid, s, name)
-                        : launch_gemm_n<EPI, 256, MB, FP8>(a, grid, s, name);
+            return pair ? launch_gemm_n<EPI, 256, MB, FP8, true>(a, grid, s, name, false, pdl)
+                        : launch_gemm_n<EPI, 256, MB, FP8>(a, grid, s, name, false, pdl);
         default: return MOE_ERR_UNSUPPORTED;
     }
 }
@@ -522,38 +562,38 @@ int32_t launch_gemm_mb(int nmax, const GemmArgs& a, int grid, cudaStream_t s, co
 // FP8 expert GEMMs: gate/up (+SwiGLU) and down with the store epilogue.
 template <int EPI>
 int32_t launch_gemm_fp8(int nmax, int mb, const GemmArgs& a, int64_t max_tiles, cudaStream_t s,
-                        const char* name) {
+                        const char* name, bool pdl = false) {
     int grid = static_cast<int>(std::min<int64_t>(sm_count(), std::max<int64_t>(1, max_tiles)));
     const bool pair = use_pair() && nmax >= 64;
     if constexpr (EPI == EPI_SWIGLU) {
-        return launch_gemm_mb<EPI, 2, true>(nmax, a, grid, s, name, pair);
+        return launch_gemm_mb<EPI, 2, true>(nmax, a, grid, s, name, pair, pdl);
     } else {
         static_assert(EPI == EPI_DOWN_STORE, "FP8 down GEMM uses the store epilogue");
-        if (mb == 2) return launch_gemm_mb<EPI, 2, true>(nmax, a, grid, s, name, pair);
-        return launch_gemm_mb<EPI, 1, true>(nmax, a, grid, s, name);
+        if (mb == 2) return launch_gemm_mb<EPI, 2, true>(nmax, a, grid, s, name, pair, pdl);
+        return launch_gemm_mb<EPI, 1, true>(nmax, a, grid, s, name, false, pdl);
     }
 }
 
 // Launch with a persistent grid of min(#SMs, tiles) CTAs.
 template <int EPI>
 int32_t launch_gemm(int nmax, int mb, const GemmArgs& a, int64_t max_tiles, cudaStream_t s,
-                    const char* name) {
+                    const char* name, bool pdl = false) {
     int grid = static_cast<int>(std::min<int64_t>(sm_count(), std::max<int64_t>(1, max_tiles)));
     if constexpr (EPI == EPI_SWIGLU) {
         if (a.gather_tok != nullptr) {
             // row gather by four dedicated gather warps
             switch (nmax) {
-                case 16: return launch_gemm_n<EPI, 16, 2, false, false, 4>(a, grid, s, name);
-                case 32: return launch_gemm_n<EPI, 32, 2, false, false, 4>(a, grid, s, name);
-                case 64: return launch_gemm_n<EPI, 64, 2, false, false, 4>(a, grid, s, name);
-                case 128: return launch_gemm_n<EPI, 128, 2, false, false, 4>(a, grid, s, name);
-                case 160: return launch_gemm_n<EPI, 160, 2, false, false, 4>(a, grid, s, name);
-                case 256: return launch_gemm_n<EPI, 256, 2, false, false, 4>(a, grid, s, name);
+                case 16: return launch_gemm_n<EPI, 16, 2, false, false, 4>(a, grid, s, name, false, pdl);
+                case 32: return launch_gemm_n<EPI, 32, 2, false, false, 4>(a, grid, s, name, false, pdl);
+                case 64: return launch_gemm_n<EPI, 64, 2, false, false, 4>(a, grid, s, name, false, pdl);
+                case 128: return launch_gemm_n<EPI, 128, 2, false, false, 4>(a, grid, s, name, false, pdl);
+                case 160: return launch_gemm_n<EPI, 160, 2, false, false, 4>(a, grid, s, name, false, pdl);
+                case 256: return launch_gemm_n<EPI, 256, 2, false, false, 4>(a, grid, s, name, false, pdl);
                 default: return MOE_ERR_UNSUPPORTED;
             }
         }
         const bool pair = use_pair() && nmax >= 64;
-        return launch_gemm_mb<EPI, 2>(nmax, a, grid, s, name, pair);
+        return launch_gemm_mb<EPI, 2>(nmax, a, grid, s, name, pair, pdl);
     } else if constexpr (EPI == EPI_LOGITS) {
         if (nmax == 256) {
             if (mb == 2) return launch_gemm_n<EPI, 256, 2>(a, grid, s, name);
@@ -568,8 +608,8 @@ int32_t launch_gemm(int nmax, int mb, const GemmArgs& a, int64_t max_tiles, cuda
         return launch_gemm_n<EPI, 32, 1>(a, grid, s, name);
     } else {
         const bool pair = EPI == EPI_DOWN_STORE && use_pair() && nmax >= 64 && mb == 2;
-        if (mb == 2) return launch_gemm_mb<EPI, 2>(nmax, a, grid, s, name, pair);
-        return launch_gemm_mb<EPI, 1>(nmax, a, grid, s, name);
+        if (mb == 2) return launch_gemm_mb<EPI, 2>(nmax, a, grid, s, name, pair, pdl);
+        return launch_gemm_mb<EPI, 1>(nmax, a, grid, s, name, false, pdl);
     }
 }
 
@@ -586,7 +626,7 @@ int64_t max_tiles(int64_t rows_total, int nseg, int nmax, int64_t m_total,
 // rows in slot order, which is deterministic and leaves the L2 atomic units
 // out of the critical path.
 bool combine_atomic() {
-    static const bool v = [] {
+    const bool v = [] {
         const char* e = std::getenv("MOE_COMBINE");
         return e && std::strcmp(e, "atomic") == 0;
     }();
@@ -599,13 +639,38 @@ bool combine_atomic() {
 // producer warp (measured 3x slower gate/up at 4096 tokens); at decode sizes
 // the two are even.
 bool fused_gather() {
-    static const bool v = env_int("MOE_FUSED_GATHER", 0) != 0;
+    const bool v = env_int("MOE_FUSED_GATHER", 0) != 0;
     return v;
 }
 
 // L2 cache hints on the GEMM operand loads (MOE_L2_HINTS=0 turns them off).
 int l2_hints() {
-    static const int v = env_int("MOE_L2_HINTS", 1) ? 1 : 0;
+    const int v = env_int("MOE_L2_HINTS", 1) ? 1 : 0;
+    return v;
+}
+
+// Rotated K order in the expert GEMMs (MOE_KROT=0 turns it off): concurrent
+// tiles start their K loops at different offsets, spreading the weight reads
+// of the CTAs over the DRAM channels instead of sweeping one column band of
+// many rows in lockstep.
+int k_rotate() {
+    const int v = env_int("MOE_KROT", 1) ? 1 : 0;
+    return v;
+}
+
+// Programmatic dependent launch along the forward's kernel chain (MOE_PDL=0
+// turns it off): each kernel may start while its predecessor finishes, does
+// its independent set-up (and, in the expert GEMMs, pulls its first weight
+// tiles into L2), then waits for the predecessor before reading its outputs.
+bool pdl_enabled() {
+    const bool v = env_int("MOE_PDL", 1) != 0;
+    return v;
+}
+
+// Weight K-steps of each CTA's first tile prefetched into L2 before the
+// dependency wait of an expert GEMM launched programmatically (MOE_PREFETCH).
+int prefetch_ksteps() {
+    const int v = std::max(0, std::min(64, env_int("MOE_PREFETCH", 8)));
     return v;
 }
 
@@ -617,6 +682,22 @@ GemmArgs base_args(int32_t* status) {
     a.l2_hints = l2_hints();
     a.status = status;
     return a;
+}
+
+// Weight read-ahead distance of the expert GEMMs in pipeline steps
+// (MOE_PF_DIST; 0 = off).
+int pf_dist() {
+    const int v = std::max(0, std::min(32, env_int("MOE_PF_DIST", 0)));
+    return v;
+}
+
+// Expert GEMM arguments for a launch that may start early (pdl): prefetch the
+// first weight tiles and let the following launch start early too.
+void expert_gemm_launch_args(GemmArgs& a, bool pdl, bool trigger_early) {
+    a.k_rotate = k_rotate();
+    a.pf_dist = pf_dist();
+    a.prefetch_ksteps = pdl ? prefetch_ksteps() : 0;
+    a.pdl_trigger_early = trigger_early ? 1 : 0;
 }
 
 // Fused routing outputs of the router GEMM (see GemmArgs::route_idx).
@@ -632,7 +713,7 @@ constexpr int kFusedRouteMaxTokens = 32;  // tokens one CTA routes in the fused 
 
 // MOE_FUSED_ROUTE=0 keeps the router GEMM and the top-k kernel separate.
 bool fused_route_enabled() {
-    static const bool v = env_int("MOE_FUSED_ROUTE", 1) != 0;
+    const bool v = env_int("MOE_FUSED_ROUTE", 1) != 0;
     return v;
 }
 
@@ -745,7 +826,8 @@ int32_t run_cast(const void* in, void* out, int64_t n, cudaStream_t s) {
 
 template <typename TIn, typename TOut>
 int32_t run_gather(const TIn* x, int64_t T, int H, int k, const int32_t* pos, int64_t n_rows,
-                   TOut* x_perm, __nv_bfloat16* x_bf16, float* acc_zero, cudaStream_t s);
+                   TOut* x_perm, __nv_bfloat16* x_bf16, float* acc_zero, cudaStream_t s,
+                   bool pdl = false);
 
 }  // namespace
 
@@ -766,6 +848,8 @@ __global__ void gather_kernel(const TIn* __restrict__ x, int64_t T, int H, int k
     const int64_t t = gw / nseg;
     if (t >= T) return;
     const int seg = static_cast<int>(gw - t * nseg);
+    ptx::grid_dep_wait();  // positions come from the previous launch
+    ptx::grid_dep_launch();
     int my_pos = -1;
     if (lane < k) {
         my_pos = pos[t * k + lane];
@@ -827,13 +911,15 @@ namespace {
 
 template <typename TIn, typename TOut>
 int32_t run_gather(const TIn* x, int64_t T, int H, int k, const int32_t* pos, int64_t n_rows,
-                   TOut* x_perm, __nv_bfloat16* x_bf16, float* acc_zero, cudaStream_t s) {
+                   TOut* x_perm, __nv_bfloat16* x_bf16, float* acc_zero, cudaStream_t s,
+                   bool pdl) {
     const int warps = 8;
     const int64_t segs = (H / (16 / static_cast<int>(sizeof(TOut))) + 32 * 8 - 1) / (32 * 8);
-    const unsigned blocks = static_cast<unsigned>((T * segs + warps - 1) / warps);
+    const int blocks = static_cast<int>((T * segs + warps - 1) / warps);
     MOE_LAUNCH("dispatch_gather", s,
-               gather_kernel<TIn, TOut><<<blocks, warps * 32, 0, s>>>(x, T, H, k, pos, n_rows,
-                                                                      x_perm, x_bf16, acc_zero));
+               if (launch_ex(gather_kernel<TIn, TOut>, blocks, warps * 32, 0, s, pdl, x, T, H, k,
+                             pos, n_rows, x_perm, x_bf16, acc_zero) != cudaSuccess)
+                   return MOE_ERR_CUDA);
     return MOE_OK;
 }
 
@@ -842,15 +928,16 @@ int32_t run_gather(const TIn* x, int64_t T, int H, int k, const int32_t* pos, in
 template <typename TOut>
 int32_t run_gather_sum(const __nv_bfloat16* y, const int32_t* pos, int64_t T, int H, int k,
                        int64_t n_rows, int64_t shared_row0, TOut* out, int32_t* status,
-                       cudaStream_t s) {
+                       cudaStream_t s, bool pdl = false) {
     const int warps = 8;
     const int64_t segs = (H / 8 + kSegVecs - 1) / kSegVecs;
-    const unsigned blocks = static_cast<unsigned>((T * segs + warps - 1) / warps);
+    const int blocks = static_cast<int>((T * segs + warps - 1) / warps);
     // two rows' loads in flight per lane before adding: measured faster than
     // wider batches, whose register use lowers the number of resident warps
     MOE_LAUNCH("combine_gather", s,
-               (gather_sum_kernel<TOut, 2><<<blocks, warps * 32, 0, s>>>(
-                   y, pos, T, H, k, n_rows, shared_row0, out, status)));
+               if (launch_ex(gather_sum_kernel<TOut, 2>, blocks, warps * 32, 0, s, pdl, y, pos, T,
+                             H, k, n_rows, shared_row0, out, status) != cudaSuccess)
+                   return MOE_ERR_CUDA);
     return MOE_OK;
 }
 
@@ -859,28 +946,30 @@ int32_t run_dispatch(const moe_problem* p, const int32_t* idx, const float* topk
                      int32_t* base, int32_t* counts, int32_t* offsets, int32_t* sched_gu,
                      int nmax_gu, int32_t* sched_dn, int nmax_dn, int32_t* pos, int32_t* src,
                      float* row_w, int32_t* status, cudaStream_t s) {
-    const unsigned nch = static_cast<unsigned>(perm_chunks(p->T));
+    const int nch = static_cast<int>(perm_chunks(p->T));
+    const bool pdl = pdl_enabled();
     MOE_LAUNCH("dispatch_count", s,
                dispatch_count_kernel<<<nch, kPermTokens, 0, s>>>(idx, p->T, p->E, p->top_k, hist,
                                                                  status));
     MOE_LAUNCH("dispatch_scan", s,
-               dispatch_scan_kernel<<<1, 512, 0, s>>>(hist, static_cast<int>(nch), p->E, p->T,
-                                                      p->top_k, p->num_shared, base, counts,
-                                                      offsets, sched_gu, nmax_gu, sched_dn,
-                                                      nmax_dn));
+               if (launch_ex(dispatch_scan_kernel, 1, 512, 0, s, pdl, hist, nch, p->E, p->T,
+                             p->top_k, p->num_shared, base, counts, offsets, sched_gu, nmax_gu,
+                             sched_dn, nmax_dn) != cudaSuccess) return MOE_ERR_CUDA);
     MOE_LAUNCH("dispatch_scatter", s,
-               dispatch_scatter_kernel<<<nch, kPermTokens, 0, s>>>(
-                   idx, topk_w, p->T, p->E, p->top_k, base, offsets, pos, src, row_w, status));
+               if (launch_ex(dispatch_scatter_kernel, nch, kPermTokens, 0, s, pdl, idx, topk_w,
+                             p->T, p->E, p->top_k, base, offsets, pos, src, row_w, status) !=
+                   cudaSuccess) return MOE_ERR_CUDA);
     return MOE_OK;
 }
 
 template <typename TOut>
-int32_t run_finalize(const float* acc, TOut* out, int64_t n, cudaStream_t s) {
+int32_t run_finalize(const float* acc, TOut* out, int64_t n, cudaStream_t s, bool pdl = false) {
     const int64_t n4 = n / 4;
-    const int64_t blocks = std::min<int64_t>((n4 + 255) / 256, 148 * 8);
+    const int blocks =
+        static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((n4 + 255) / 256, 148 * 8)));
     MOE_LAUNCH("finalize", s,
-               finalize_kernel<TOut><<<static_cast<unsigned>(std::max<int64_t>(1, blocks)), 256, 0,
-                                       s>>>(acc, out, n4));
+               if (launch_ex(finalize_kernel<TOut>, blocks, 256, 0, s, pdl, acc, out, n4) !=
+                   cudaSuccess) return MOE_ERR_CUDA);
     return MOE_OK;
 }
 
@@ -921,6 +1010,15 @@ size_t moe_workspace_size(const moe_problem* p, int32_t call) {
         return layout_for(p, call, rows, p->E).total;
     }
     return layout_for(p, call).total;
+}
+
+int32_t moe_expert_tile_rows(const moe_problem* p, int32_t* gate_up_rows, int32_t* down_rows) {
+    MOE_TRY(check_problem(p));
+    if (!gate_up_rows || !down_rows) return MOE_ERR_INVALID_ARG;
+    const int nmax = pick_nmax(static_cast<double>(p->T * p->top_k) / p->E);
+    *gate_up_rows = nmax;
+    *down_rows = pick_down_nmax(nmax);
+    return MOE_OK;
 }
 
 int32_t moe_router_logits(const moe_problem* p, const void* x, const void* gate_w, float* logits,
@@ -1029,6 +1127,9 @@ int32_t moe_grouped_swiglu_ffn(const moe_problem* p, const void* x_perm, int64_t
         a.out = h;
         a.out_ld = static_cast<int32_t>(I);
         a.clip = effective_clip(p);
+        // an ordinary launch: the schedule it reads first is the previous
+        // launch's output; the down GEMM may start as soon as it is resident
+        expert_gemm_launch_args(a, false, true);
         MOE_TRY(launch_gemm<EPI_SWIGLU>(nmax, 2, a, max_tiles(rows, n_groups, nmax, I), s,
                                         "expert_gate_up_gemm"));
     }
@@ -1049,9 +1150,11 @@ int32_t moe_grouped_swiglu_ffn(const moe_problem* p, const void* x_perm, int64_t
         a.out = y_perm;
         a.out_ld = static_cast<int32_t>(H);
         a.out_f32 = p->dtype == MOE_F32 ? 1 : 0;
+        const bool pdl = pdl_enabled();
+        expert_gemm_launch_args(a, pdl, false);
         MOE_TRY(launch_gemm<EPI_DOWN_STORE>(nmax, mb, a,
                                             max_tiles(rows, n_groups, nmax, H, 128 * mb), s,
-                                            "expert_down_gemm"));
+                                            "expert_down_gemm", pdl));
     }
     return MOE_OK;
 }
@@ -1139,6 +1242,10 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
     //    GEMM (from x, by src); fp32 problems copy them into x_perm as bf16.
     //    The scatter-add combine also needs its fp32 accumulator zeroed.
     __nv_bfloat16* x_perm = at<__nv_bfloat16>(ws, L.x_perm);
+    // launches from here on may start while their predecessor finishes: each
+    // waits for it before reading its outputs, and reads nothing earlier than
+    // that except what was complete before the predecessor could start
+    const bool pdl = pdl_enabled();
     const bool atomic_combine = combine_atomic();
     float* out_acc = atomic_combine ? at<float>(ws, L.out_acc) : nullptr;
     __nv_bfloat16* y_perm = at<__nv_bfloat16>(ws, L.y_perm);
@@ -1147,12 +1254,12 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
     if (f32) {
         MOE_TRY((run_gather<float, __nv_bfloat16>(static_cast<const float*>(x), T, p->H, p->top_k,
                                                   pos, T * k, x_perm, at<__nv_bfloat16>(ws, L.x_bf16),
-                                                  out_acc, s)));
+                                                  out_acc, s, pdl)));
         x_b = at<void>(ws, L.x_bf16);
     } else if (!gather_in_gemm) {
         MOE_TRY((run_gather<__nv_bfloat16, __nv_bfloat16>(static_cast<const __nv_bfloat16*>(x), T,
                                                           p->H, p->top_k, pos, T * k, x_perm,
-                                                          nullptr, out_acc, s)));
+                                                          nullptr, out_acc, s, pdl)));
     } else if (out_acc) {
         if (cudaMemsetAsync(out_acc, 0, static_cast<size_t>(T) * H * sizeof(float), s) !=
             cudaSuccess)
@@ -1189,8 +1296,12 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
             a.gather_src = x;
             a.n_tokens = static_cast<int32_t>(T);
         }
+        // (after a memset, the scatter-add mode's fused-gather form, the
+        // launch is an ordinary one)
+        const bool pdl_gu = pdl && !(gather_in_gemm && out_acc);
+        expert_gemm_launch_args(a, pdl_gu, true);
         MOE_TRY(launch_gemm<EPI_SWIGLU>(nmax, 2, a, max_tiles(h_rows, nseg, nmax, I), s,
-                                        "expert_gate_up_gemm"));
+                                        "expert_gate_up_gemm", pdl_gu));
     }
     // 5. grouped down GEMM; its epilogue applies the routing weight and either
     //    stores the weighted rows (gather combine) or scatter-adds them into the
@@ -1219,26 +1330,29 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
         a.row_weight = row_w;
         a.routed_rows = static_cast<int32_t>(T * k);
         const int64_t tiles = max_tiles(h_rows, nseg, nmax_dn, H, 128 * mb);
+        expert_gemm_launch_args(a, pdl, false);
         if (atomic_combine) {
             a.out = out_acc;
             MOE_TRY(launch_gemm<EPI_DOWN_ATOMIC>(nmax_dn, mb, a, tiles, s,
-                                                 "expert_down_combine_gemm"));
+                                                 "expert_down_combine_gemm", pdl));
         } else {
             a.out = y_perm;
-            MOE_TRY(launch_gemm<EPI_DOWN_STORE>(nmax_dn, mb, a, tiles, s, "expert_down_gemm"));
+            MOE_TRY(launch_gemm<EPI_DOWN_STORE>(nmax_dn, mb, a, tiles, s, "expert_down_gemm",
+                                                pdl));
         }
     }
     // 6. token-order output
     if (atomic_combine) {
-        if (f32) return run_finalize<float>(out_acc, static_cast<float*>(out), T * H, s);
-        return run_finalize<__nv_bfloat16>(out_acc, static_cast<__nv_bfloat16*>(out), T * H, s);
+        if (f32) return run_finalize<float>(out_acc, static_cast<float*>(out), T * H, s, pdl);
+        return run_finalize<__nv_bfloat16>(out_acc, static_cast<__nv_bfloat16*>(out), T * H, s,
+                                           pdl);
     }
     const int64_t shared_row0 = S ? T * k : -1;
     if (f32)
         return run_gather_sum(y_perm, pos, T, p->H, p->top_k, T * k, shared_row0,
-                              static_cast<float*>(out), status, s);
+                              static_cast<float*>(out), status, s, pdl);
     return run_gather_sum(y_perm, pos, T, p->H, p->top_k, T * k, shared_row0,
-                          static_cast<__nv_bfloat16*>(out), status, s);
+                          static_cast<__nv_bfloat16*>(out), status, s, pdl);
 }
 
 }  // extern "C"
@@ -1405,8 +1519,9 @@ int32_t moe_forward_fp8(const moe_problem* p, const void* x, const void* gate_w,
                                                           0, s>>>(
                    static_cast<const __nv_bfloat16*>(x), T, static_cast<int>(H), T, T, x_q, s_x));
     uint8_t* x_perm = at<uint8_t>(ws, L.x_perm);
+    const bool pdl = pdl_enabled();
     MOE_TRY((run_gather<uint8_t, uint8_t>(x_q, T, p->H, p->top_k, pos, T * k, x_perm, nullptr,
-                                          nullptr, s)));
+                                          nullptr, s, pdl)));
     // 4. gate/up on E4M3 codes; the epilogue applies token x channel scales,
     //    clamps, and writes h as E4M3 with the fixed power-of-two scale
     const double L_clip = p->clip_limit;
@@ -1444,8 +1559,9 @@ int32_t moe_forward_fp8(const moe_problem* p, const void* x, const void* gate_w,
         a.scale_w_special = shared_s_gu;
         a.h_scale = h_scale;
         a.h_scale_inv = 1.0f / h_scale;
+        expert_gemm_launch_args(a, pdl, true);
         MOE_TRY(launch_gemm_fp8<EPI_SWIGLU>(nmax, 2, a, max_tiles(h_rows, nseg, nmax, I), s,
-                                            "expert_gate_up_gemm_fp8"));
+                                            "expert_gate_up_gemm_fp8", pdl));
     }
     // 5. down on E4M3 codes; epilogue: h scale x column scale x routing weight
     __nv_bfloat16* y_perm = at<__nv_bfloat16>(ws, L.y_perm);
@@ -1477,13 +1593,14 @@ int32_t moe_forward_fp8(const moe_problem* p, const void* x, const void* gate_w,
         a.scale_w_special = shared_s_d;
         a.h_scale = h_scale;
         a.h_scale_inv = 1.0f / h_scale;
+        expert_gemm_launch_args(a, pdl, false);
         MOE_TRY(launch_gemm_fp8<EPI_DOWN_STORE>(nmax_dn, mb, a,
                                                 max_tiles(h_rows, nseg, nmax_dn, H, 128 * mb), s,
-                                                "expert_down_gemm_fp8"));
+                                                "expert_down_gemm_fp8", pdl));
     }
     // 6. fixed-order combine into token order
     return run_gather_sum(y_perm, pos, T, p->H, p->top_k, T * k, S ? T * k : -1,
-                          static_cast<__nv_bfloat16*>(out), status, s);
+                          static_cast<__nv_bfloat16*>(out), status, s, pdl);
 }
 
 int32_t moe_read_device_status(const void* ws, int32_t* status_out, void* stream) {

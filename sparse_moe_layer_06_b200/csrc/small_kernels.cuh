@@ -229,6 +229,8 @@ __global__ void __launch_bounds__(512) dispatch_scan_kernel(
     int32_t* sched_gu, int nmax_gu, int32_t* sched_dn, int nmax_dn) {
     __shared__ int s_warp[32];
     const int tid = threadIdx.x;
+    ptx::grid_dep_wait();  // the histogram comes from the previous launch
+    ptx::grid_dep_launch();
     int cnt = 0;
     if (tid < E) {
         int running = 0;
@@ -290,6 +292,8 @@ __global__ void dispatch_scatter_kernel(const int32_t* __restrict__ idx,
     __shared__ int32_t wbase[kPermWarps][kMaxExperts];
     for (int i = threadIdx.x; i < kPermWarps * kMaxExperts; i += blockDim.x)
         (&masks[0][0])[i] = 0u;
+    ptx::grid_dep_wait();  // bases and offsets come from the previous launch
+    ptx::grid_dep_launch();
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t = static_cast<int64_t>(blockIdx.x) * kPermTokens + threadIdx.x;
@@ -361,6 +365,7 @@ __global__ void schedule_from_offsets_kernel(const int32_t* __restrict__ offsets
 // out[t,h] = cast(acc[t,h]), 4 elements per thread.
 template <typename TOut>
 __global__ void finalize_kernel(const float* __restrict__ acc, TOut* __restrict__ out, int64_t n4) {
+    ptx::grid_dep_wait();  // the accumulator comes from the previous launch
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const float4 v = reinterpret_cast<const float4*>(acc)[i];
@@ -435,6 +440,7 @@ __global__ void gather_sum_kernel(const __nv_bfloat16* __restrict__ y,
     const int lane = threadIdx.x & 31;
     const int nvec = H / 8;
     const int nseg = (nvec + kSegVecs - 1) / kSegVecs;
+    ptx::grid_dep_wait();  // the rows come from the previous launch
     const int64_t gw = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int64_t t = gw / nseg;
     if (t >= T) return;

@@ -2,7 +2,9 @@
 
 Every function here has the name of the C entry point it calls and does no
 arithmetic of its own: it checks that the torch tensors it is handed are CUDA,
-contiguous and of the expected dtype, passes their device pointers and the
+contiguous, of the expected dtype and at least as large as the problem needs
+(the kernels take their extents from the problem, so a short tensor would be
+accessed out of bounds on the device), passes their device pointers and the
 current CUDA stream to the library, and raises if the library returns an error.
 PyTorch only supplies device memory and streams.
 
@@ -32,7 +34,7 @@ EXPORTED = (
     "moe_grouped_swiglu_ffn", "moe_combine", "moe_forward", "moe_read_device_status",
     "moe_clear_device_status", "moe_launch_count", "moe_profile_start", "moe_profile_stop",
     "moe_route_noalloc", "moe_router_stats", "moe_quantize_weights_fp8", "moe_forward_fp8",
-    "moe_check_wait_timeout",
+    "moe_check_wait_timeout", "moe_expert_tile_rows",
 )
 ROUTE_NOALLOC_SCRATCH_BYTES = 1 << 20
 
@@ -117,6 +119,7 @@ def load_library(path: str = LIB_PATH):
             "moe_quantize_weights_fp8": (I32, [PP, I32, P, P, P, P, P]),
             "moe_forward_fp8": (I32, [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]),
             "moe_check_wait_timeout": (I32, [P, SZ, ctypes.POINTER(I32), P]),
+            "moe_expert_tile_rows": (I32, [PP, ctypes.POINTER(I32), ctypes.POINTER(I32)]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -136,18 +139,45 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _ptr(t, dtype=None, name="tensor", optional=False):
-    if t is None:
-        if optional:
-            return None
-        raise ValueError(f"{name} is required")
-    if not isinstance(t, torch.Tensor) or not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor")
-    if not t.is_contiguous():
-        raise ValueError(f"{name} must be contiguous")
-    if dtype is not None and t.dtype != dtype:
-        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
-    return ctypes.c_void_p(t.data_ptr())
+def _ptr(t, dtype=None, name="tensor", optional=False, numel=None):
+    """Device pointer of `t` after checking it: a contiguous CUDA tensor of
+    `dtype` holding at least `numel` elements (the kernels take their extents
+    from the problem, not from the tensor, so a short tensor would be read or
+    written out of bounds on the device)."""
+    return _ptrs((t, dtype, name, optional, numel))[0]
+
+
+def _ptrs(*specs):
+    """Pointers of several operands, each spec (tensor, dtype, name, optional,
+    numel).  Every operand's type, dtype, size and layout is checked before
+    any operand's device, so the first error names the operand that is
+    actually wrong."""
+    for t, dtype, name, optional, numel in specs:
+        if t is None:
+            if optional:
+                continue
+            raise ValueError(f"{name} is required")
+        if not isinstance(t, torch.Tensor):
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if dtype is not None and t.dtype != dtype:
+            raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+        if numel is not None and t.numel() < numel:
+            raise ValueError(f"{name} has {t.numel()} elements, the problem needs {numel}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    out = []
+    for t, _, name, _, _ in specs:
+        if t is None:
+            out.append(None)
+            continue
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        out.append(ctypes.c_void_p(t.data_ptr()))
+    return out
+
+
+def _spec(t, dtype=None, name="tensor", optional=False, numel=None):
+    return (t, dtype, name, optional, numel)
 
 
 def _check(status: int, what: str):
@@ -170,21 +200,34 @@ def alloc_workspace(problem: MoEProblem, call: int, device=None, extra: int = 0)
     return ws
 
 
+def _ws(workspace):
+    return _spec(workspace, None, "workspace")
+
+
 def moe_router_logits(problem, x, gate_w, logits, workspace, stream=None):
     pc = problem.c()
-    _check(load_library().moe_router_logits(
-        ctypes.byref(pc), _ptr(x, problem.dtype, "x"), _ptr(gate_w, problem.dtype, "gate_w"),
-        _ptr(logits, torch.float32, "logits"), _ptr(workspace, None, "workspace"),
-        workspace.numel(), _stream(stream)), "moe_router_logits")
+    T, H, E = problem.T, problem.H, problem.E
+    ptrs = _ptrs(_spec(x, problem.dtype, "x", numel=T * H),
+                 _spec(gate_w, problem.dtype, "gate_w", numel=E * H),
+                 _spec(logits, torch.float32, "logits", numel=T * E), _ws(workspace))
+    _check(load_library().moe_router_logits(ctypes.byref(pc), *ptrs, workspace.numel(),
+                                            _stream(stream)), "moe_router_logits")
+
+
+def _route_specs(problem, x, gate_w, logit_bias, topk_idx, topk_w):
+    T, H, E, k = problem.T, problem.H, problem.E, problem.top_k
+    return (_spec(x, problem.dtype, "x", numel=T * H),
+            _spec(gate_w, problem.dtype, "gate_w", numel=E * H),
+            _spec(logit_bias, torch.float32, "logit_bias", optional=True, numel=E),
+            _spec(topk_idx, torch.int32, "topk_idx", numel=T * k),
+            _spec(topk_w, torch.float32, "topk_w", numel=T * k))
 
 
 def moe_route(problem, x, gate_w, logit_bias, topk_idx, topk_w, workspace, stream=None):
     pc = problem.c()
-    _check(load_library().moe_route(
-        ctypes.byref(pc), _ptr(x, problem.dtype, "x"), _ptr(gate_w, problem.dtype, "gate_w"),
-        _ptr(logit_bias, torch.float32, "logit_bias", optional=True),
-        _ptr(topk_idx, torch.int32, "topk_idx"), _ptr(topk_w, torch.float32, "topk_w"),
-        _ptr(workspace, None, "workspace"), workspace.numel(), _stream(stream)), "moe_route")
+    ptrs = _ptrs(*_route_specs(problem, x, gate_w, logit_bias, topk_idx, topk_w), _ws(workspace))
+    _check(load_library().moe_route(ctypes.byref(pc), *ptrs, workspace.numel(), _stream(stream)),
+           "moe_route")
 
 
 def moe_route_noalloc(problem, x, gate_w, logit_bias, topk_idx, topk_w, stream=None):
@@ -194,53 +237,62 @@ def moe_route_noalloc(problem, x, gate_w, logit_bias, topk_idx, topk_w, stream=N
     device array inside the library; T*E*4 + 256 bytes must fit in it.
     Calls that overlap on the GPU race on that array."""
     pc = problem.c()
-    _check(load_library().moe_route_noalloc(
-        ctypes.byref(pc), _ptr(x, problem.dtype, "x"), _ptr(gate_w, problem.dtype, "gate_w"),
-        _ptr(logit_bias, torch.float32, "logit_bias", optional=True),
-        _ptr(topk_idx, torch.int32, "topk_idx"), _ptr(topk_w, torch.float32, "topk_w"),
-        _stream(stream)), "moe_route_noalloc")
+    ptrs = _ptrs(*_route_specs(problem, x, gate_w, logit_bias, topk_idx, topk_w))
+    _check(load_library().moe_route_noalloc(ctypes.byref(pc), *ptrs, _stream(stream)),
+           "moe_route_noalloc")
 
 
 def moe_router_stats(problem, x, gate_w, logit_bias, P_out, f_out, aux_out, ema_counts,
                      ema_total, momentum, workspace, stream=None):
     pc = problem.c()
-    _check(load_library().moe_router_stats(
-        ctypes.byref(pc), _ptr(x, problem.dtype, "x"), _ptr(gate_w, problem.dtype, "gate_w"),
-        _ptr(logit_bias, torch.float32, "logit_bias", optional=True),
-        _ptr(P_out, torch.float32, "P_out"), _ptr(f_out, torch.float32, "f_out"),
-        _ptr(aux_out, torch.float32, "aux_out"),
-        _ptr(ema_counts, torch.float32, "ema_counts", optional=True),
-        _ptr(ema_total, torch.float32, "ema_total", optional=True), float(momentum),
-        _ptr(workspace, None, "workspace"), workspace.numel(), _stream(stream)),
-        "moe_router_stats")
+    T, H, E = problem.T, problem.H, problem.E
+    ptrs = _ptrs(_spec(x, problem.dtype, "x", numel=T * H),
+                 _spec(gate_w, problem.dtype, "gate_w", numel=E * H),
+                 _spec(logit_bias, torch.float32, "logit_bias", optional=True, numel=E),
+                 _spec(P_out, torch.float32, "P_out", numel=E),
+                 _spec(f_out, torch.float32, "f_out", numel=E),
+                 _spec(aux_out, torch.float32, "aux_out", numel=1),
+                 _spec(ema_counts, torch.float32, "ema_counts", optional=True, numel=E),
+                 _spec(ema_total, torch.float32, "ema_total", optional=True, numel=1),
+                 _ws(workspace))
+    _check(load_library().moe_router_stats(ctypes.byref(pc), *ptrs[:8], float(momentum),
+                                           ptrs[8], workspace.numel(), _stream(stream)),
+           "moe_router_stats")
 
 
 def moe_quantize_weights_fp8(problem, w, q, scale_gu, scale_d, stream=None):
     """Encode [n,3,I,H] weights into E4M3 codes q (uint8, same shape) with
     scale_gu [n,2,I] and scale_d [n,H] (fp32); n is w.shape[0]."""
     pc = problem.c()
-    _check(load_library().moe_quantize_weights_fp8(
-        ctypes.byref(pc), int(w.shape[0]), _ptr(w, problem.dtype, "w"),
-        _ptr(q, torch.uint8, "q"), _ptr(scale_gu, torch.float32, "scale_gu"),
-        _ptr(scale_d, torch.float32, "scale_d"), _stream(stream)), "moe_quantize_weights_fp8")
+    n, H, I = int(w.shape[0]), problem.H, problem.I
+    ptrs = _ptrs(_spec(w, problem.dtype, "w", numel=n * 3 * I * H),
+                 _spec(q, torch.uint8, "q", numel=n * 3 * I * H),
+                 _spec(scale_gu, torch.float32, "scale_gu", numel=n * 2 * I),
+                 _spec(scale_d, torch.float32, "scale_d", numel=n * H))
+    _check(load_library().moe_quantize_weights_fp8(ctypes.byref(pc), n, *ptrs, _stream(stream)),
+           "moe_quantize_weights_fp8")
 
 
 def moe_forward_fp8(problem, x, gate_w, logit_bias, expert_q, expert_s_gu, expert_s_d,
                     shared_q, shared_s_gu, shared_s_d, out, topk_idx_out, topk_w_out, workspace,
                     stream=None):
     pc = problem.c()
-    _check(load_library().moe_forward_fp8(
-        ctypes.byref(pc), _ptr(x, torch.bfloat16, "x"), _ptr(gate_w, torch.bfloat16, "gate_w"),
-        _ptr(logit_bias, torch.float32, "logit_bias", optional=True),
-        _ptr(expert_q, torch.uint8, "expert_q"), _ptr(expert_s_gu, torch.float32, "expert_s_gu"),
-        _ptr(expert_s_d, torch.float32, "expert_s_d"),
-        _ptr(shared_q, torch.uint8, "shared_q", optional=True),
-        _ptr(shared_s_gu, torch.float32, "shared_s_gu", optional=True),
-        _ptr(shared_s_d, torch.float32, "shared_s_d", optional=True),
-        _ptr(out, torch.bfloat16, "out"),
-        _ptr(topk_idx_out, torch.int32, "topk_idx_out", optional=True),
-        _ptr(topk_w_out, torch.float32, "topk_w_out", optional=True),
-        _ptr(workspace, None, "workspace"), workspace.numel(), _stream(stream)), "moe_forward_fp8")
+    T, H, E, I, k = problem.T, problem.H, problem.E, problem.I, problem.top_k
+    ptrs = _ptrs(_spec(x, torch.bfloat16, "x", numel=T * H),
+                 _spec(gate_w, torch.bfloat16, "gate_w", numel=E * H),
+                 _spec(logit_bias, torch.float32, "logit_bias", optional=True, numel=E),
+                 _spec(expert_q, torch.uint8, "expert_q", numel=E * 3 * I * H),
+                 _spec(expert_s_gu, torch.float32, "expert_s_gu", numel=E * 2 * I),
+                 _spec(expert_s_d, torch.float32, "expert_s_d", numel=E * H),
+                 _spec(shared_q, torch.uint8, "shared_q", optional=True, numel=3 * I * H),
+                 _spec(shared_s_gu, torch.float32, "shared_s_gu", optional=True, numel=2 * I),
+                 _spec(shared_s_d, torch.float32, "shared_s_d", optional=True, numel=H),
+                 _spec(out, torch.bfloat16, "out", numel=T * H),
+                 _spec(topk_idx_out, torch.int32, "topk_idx_out", optional=True, numel=T * k),
+                 _spec(topk_w_out, torch.float32, "topk_w_out", optional=True, numel=T * k),
+                 _ws(workspace))
+    _check(load_library().moe_forward_fp8(ctypes.byref(pc), *ptrs, workspace.numel(),
+                                          _stream(stream)), "moe_forward_fp8")
 
 
 def moe_check_wait_timeout(workspace, stream=None) -> int:
@@ -255,22 +307,32 @@ def moe_check_wait_timeout(workspace, stream=None) -> int:
 
 def moe_permute(problem, topk_idx, x, offsets, pos, src_token, x_perm, workspace, stream=None):
     pc = problem.c()
-    _check(load_library().moe_permute(
-        ctypes.byref(pc), _ptr(topk_idx, torch.int32, "topk_idx"), _ptr(x, problem.dtype, "x"),
-        _ptr(offsets, torch.int32, "offsets"), _ptr(pos, torch.int32, "pos"),
-        _ptr(src_token, torch.int32, "src_token"), _ptr(x_perm, problem.dtype, "x_perm"),
-        _ptr(workspace, None, "workspace"), workspace.numel(), _stream(stream)), "moe_permute")
+    T, H, E, k = problem.T, problem.H, problem.E, problem.top_k
+    ptrs = _ptrs(_spec(topk_idx, torch.int32, "topk_idx", numel=T * k),
+                 _spec(x, problem.dtype, "x", numel=T * H),
+                 _spec(offsets, torch.int32, "offsets", numel=E + 1),
+                 _spec(pos, torch.int32, "pos", numel=T * k),
+                 _spec(src_token, torch.int32, "src_token", numel=T * k),
+                 _spec(x_perm, problem.dtype, "x_perm", numel=T * k * H), _ws(workspace))
+    _check(load_library().moe_permute(ctypes.byref(pc), *ptrs, workspace.numel(),
+                                      _stream(stream)), "moe_permute")
 
 
 def moe_grouped_swiglu_ffn(problem, x_perm, offsets, n_groups, expert_w, y_perm, workspace,
                            stream=None):
     pc = problem.c()
-    _check(load_library().moe_grouped_swiglu_ffn(
-        ctypes.byref(pc), _ptr(x_perm, problem.dtype, "x_perm"), x_perm.shape[0],
-        _ptr(offsets, torch.int32, "offsets"), int(n_groups),
-        _ptr(expert_w, problem.dtype, "expert_w"), _ptr(y_perm, problem.dtype, "y_perm"),
-        _ptr(workspace, None, "workspace"), workspace.numel(), _stream(stream)),
-        "moe_grouped_swiglu_ffn")
+    H, I, g = problem.H, problem.I, int(n_groups)
+    if not isinstance(x_perm, torch.Tensor) or x_perm.dim() != 2 or x_perm.shape[1] != H:
+        raise ValueError(f"x_perm must be a [rows, {H}] tensor")
+    rows = int(x_perm.shape[0])
+    ptrs = _ptrs(_spec(x_perm, problem.dtype, "x_perm"),
+                 _spec(offsets, torch.int32, "offsets", numel=max(0, g) + 1),
+                 _spec(expert_w, problem.dtype, "expert_w", numel=max(0, g) * 3 * I * H),
+                 _spec(y_perm, problem.dtype, "y_perm", numel=rows * H), _ws(workspace))
+    x_p, off_p, w_p, y_p, ws_p = ptrs
+    _check(load_library().moe_grouped_swiglu_ffn(ctypes.byref(pc), x_p, rows, off_p, g, w_p, y_p,
+                                                 ws_p, workspace.numel(), _stream(stream)),
+           "moe_grouped_swiglu_ffn")
 
 
 def ffn_workspace_size(problem: MoEProblem, rows: int, n_groups: int) -> int:
@@ -283,25 +345,40 @@ def ffn_workspace_size(problem: MoEProblem, rows: int, n_groups: int) -> int:
 
 def moe_combine(problem, y_perm, pos, topk_w, shared_y, out, workspace, stream=None):
     pc = problem.c()
-    _check(load_library().moe_combine(
-        ctypes.byref(pc), _ptr(y_perm, problem.dtype, "y_perm"), _ptr(pos, torch.int32, "pos"),
-        _ptr(topk_w, torch.float32, "topk_w"),
-        _ptr(shared_y, problem.dtype, "shared_y", optional=True), _ptr(out, problem.dtype, "out"),
-        _ptr(workspace, None, "workspace"), workspace.numel(), _stream(stream)), "moe_combine")
+    T, H, k = problem.T, problem.H, problem.top_k
+    ptrs = _ptrs(_spec(y_perm, problem.dtype, "y_perm", numel=T * k * H),
+                 _spec(pos, torch.int32, "pos", numel=T * k),
+                 _spec(topk_w, torch.float32, "topk_w", numel=T * k),
+                 _spec(shared_y, problem.dtype, "shared_y", optional=True, numel=T * H),
+                 _spec(out, problem.dtype, "out", numel=T * H), _ws(workspace))
+    _check(load_library().moe_combine(ctypes.byref(pc), *ptrs, workspace.numel(),
+                                      _stream(stream)), "moe_combine")
 
 
 def moe_forward(problem, x, gate_w, logit_bias, expert_w, shared_w, out, topk_idx_out,
                 topk_w_out, workspace, stream=None):
     pc = problem.c()
-    _check(load_library().moe_forward(
-        ctypes.byref(pc), _ptr(x, problem.dtype, "x"), _ptr(gate_w, problem.dtype, "gate_w"),
-        _ptr(logit_bias, torch.float32, "logit_bias", optional=True),
-        _ptr(expert_w, problem.dtype, "expert_w"),
-        _ptr(shared_w, problem.dtype, "shared_w", optional=True),
-        _ptr(out, problem.dtype, "out"),
-        _ptr(topk_idx_out, torch.int32, "topk_idx_out", optional=True),
-        _ptr(topk_w_out, torch.float32, "topk_w_out", optional=True),
-        _ptr(workspace, None, "workspace"), workspace.numel(), _stream(stream)), "moe_forward")
+    T, H, E, I, k = problem.T, problem.H, problem.E, problem.I, problem.top_k
+    ptrs = _ptrs(_spec(x, problem.dtype, "x", numel=T * H),
+                 _spec(gate_w, problem.dtype, "gate_w", numel=E * H),
+                 _spec(logit_bias, torch.float32, "logit_bias", optional=True, numel=E),
+                 _spec(expert_w, problem.dtype, "expert_w", numel=E * 3 * I * H),
+                 _spec(shared_w, problem.dtype, "shared_w", optional=True, numel=3 * I * H),
+                 _spec(out, problem.dtype, "out", numel=T * H),
+                 _spec(topk_idx_out, torch.int32, "topk_idx_out", optional=True, numel=T * k),
+                 _spec(topk_w_out, torch.float32, "topk_w_out", optional=True, numel=T * k),
+                 _ws(workspace))
+    _check(load_library().moe_forward(ctypes.byref(pc), *ptrs, workspace.numel(),
+                                      _stream(stream)), "moe_forward")
+
+
+def moe_expert_tile_rows(problem) -> tuple[int, int]:
+    """(gate/up, down) token-row tile widths of the expert GEMMs for `problem`."""
+    pc = problem.c()
+    gu, dn = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(load_library().moe_expert_tile_rows(ctypes.byref(pc), ctypes.byref(gu),
+                                                ctypes.byref(dn)), "moe_expert_tile_rows")
+    return int(gu.value), int(dn.value)
 
 
 def moe_read_device_status(workspace, stream=None) -> int:

@@ -92,3 +92,42 @@ def forward_parity(inp: dict, cfg, gpu_out: torch.Tensor, gpu_idx: torch.Tensor,
                               tokens=[tok[i] for i in exempt], forced_idx=forced)
         assert_close_out(out[exempt], ref2["out"], f"{cfg.name} near-tie rows", OUT_TOL)
     return len(exempt), err, scale
+
+
+def chunk_bounds(rows: int, width: int):
+    """[first, last] row of every token chunk of a segment of `rows` rows cut
+    for tile width `width` (the rule moe_expert_tile_rows documents:
+    c = ceil(rows / width) chunks of ceil16(ceil(rows / c)) rows)."""
+    if rows <= 0:
+        return []
+    c = -(-rows // width)
+    cl = (-(-rows // c) + 15) // 16 * 16
+    return [(i * cl, min(rows, (i + 1) * cl) - 1) for i in range(c)]
+
+
+def schedule_cover_tokens(idx: np.ndarray, E: int, num_shared: int, widths):
+    """Tokens whose output rows cover every token tile of the expert GEMMs.
+
+    The permuted rows of expert e are the tokens routed to it in ascending
+    order (the dispatch orders rows by expert, then token); the shared
+    expert's rows are all T tokens in order.  For each tile width in `widths`
+    (gate/up and down), every chunk of every segment contributes its first and
+    last row's token.  Checking a token's full output row covers all weight
+    blocks of the tiles its rows belong to.  Returns (sorted tokens,
+    {width: number of tiles}) -- every tile has at least one checked row."""
+    T = idx.shape[0]
+    by_expert = [[] for _ in range(E)]
+    for t in range(T):
+        for e in idx[t]:
+            by_expert[int(e)].append(t)
+    segments = by_expert + ([list(range(T))] if num_shared else [])
+    chosen, tiles = set(), {}
+    for width in set(widths):
+        n_tiles = 0
+        for rows in segments:
+            for first, last in chunk_bounds(len(rows), width):
+                chosen.add(rows[first])
+                chosen.add(rows[last])
+                n_tiles += 1
+        tiles[width] = n_tiles
+    return sorted(chosen), tiles

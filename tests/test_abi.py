@@ -168,3 +168,86 @@ def test_header_compiles_as_c_and_links(lib, tmp_path):
     assert r.returncode == 0, r.stderr
     r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout + r.stderr
+
+
+def test_binding_refuses_tensors_smaller_than_the_problem(lib):
+    # The kernels take every extent from the problem, so the binding must
+    # refuse an operand with fewer elements than the problem implies before
+    # the C call (on CPU tensors the size check comes before the device check).
+    p = problem(T=64, H=256, E=16, I=128, top_k=2, num_shared=1)
+    T, H, E, I, k = p.T, p.H, p.E, p.I, p.top_k
+    bf = torch.bfloat16
+    full = dict(x=torch.zeros(T, H, dtype=bf), gate_w=torch.zeros(E, H, dtype=bf),
+                expert_w=torch.zeros(E, 3, I, H, dtype=bf),
+                shared_w=torch.zeros(3, I, H, dtype=bf), out=torch.zeros(T, H, dtype=bf),
+                idx=torch.zeros(T, k, dtype=torch.int32), w=torch.zeros(T, k))
+    before = moe.moe_launch_count()
+    for name in full:
+        args = dict(full)
+        args[name] = args[name].reshape(-1)[:-1]  # one element short
+        with pytest.raises(ValueError, match="elements"):
+            moe.moe_forward(p, args["x"], args["gate_w"], None, args["expert_w"],
+                            args["shared_w"], args["out"], args["idx"], args["w"],
+                            torch.zeros(256, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="elements"):
+        moe.moe_route(p, full["x"], full["gate_w"], torch.zeros(E - 1), full["idx"], full["w"],
+                      torch.zeros(256, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="elements"):
+        moe.moe_permute(p, full["idx"], full["x"], torch.zeros(E, dtype=torch.int32),
+                        torch.zeros(T * k, dtype=torch.int32),
+                        torch.zeros(T * k, dtype=torch.int32),
+                        torch.zeros(T * k, H, dtype=bf), torch.zeros(256, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="elements"):
+        moe.moe_combine(p, torch.zeros(T * k - 1, H, dtype=bf),
+                        torch.zeros(T * k, dtype=torch.int32), full["w"], None, full["out"],
+                        torch.zeros(256, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="elements"):
+        moe.moe_grouped_swiglu_ffn(p, torch.zeros(10, H, dtype=bf),
+                                   torch.zeros(E + 1, dtype=torch.int32), E,
+                                   full["expert_w"], torch.zeros(9, H, dtype=bf),
+                                   torch.zeros(256, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="elements"):
+        moe.moe_forward_fp8(p, full["x"], full["gate_w"], None,
+                            torch.zeros(E * 3 * I * H, dtype=torch.uint8),
+                            torch.zeros(E * 2 * I), torch.zeros(E * H - 1),
+                            None, None, None, full["out"], None, None,
+                            torch.zeros(256, dtype=torch.uint8))
+    assert moe.moe_launch_count() == before
+
+
+def test_expert_tile_rows_query(lib):
+    # host-only query of the token-tile widths of the expert GEMMs
+    expect = {"tiny": 16, "hy3": 160, "hy4_prefill": 160, "hy4_decode": 16, "hy4_skew": 256}
+    for name, width in expect.items():
+        gu, dn = moe.moe_expert_tile_rows(moe.MoEProblem.from_config(CONFIGS[name]))
+        assert (gu, dn) == (width, width), name
+    with pytest.raises(moe.MoEError):
+        moe.moe_expert_tile_rows(problem(H=100))
+
+
+def test_schedule_cover_tokens_covers_every_chunk():
+    import sys
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import numpy as np
+    from parity_util import chunk_bounds, schedule_cover_tokens
+    for rows in (1, 15, 16, 17, 100, 160, 161, 320, 321, 16232):
+        for width in (16, 32, 160, 256):
+            b = chunk_bounds(rows, width)
+            # contiguous, complete, at most `width` rows, multiples of 16 but the last
+            assert b[0][0] == 0 and b[-1][1] == rows - 1
+            for (f0, l0), (f1, _) in zip(b, b[1:]):
+                assert f1 == l0 + 1 and (l0 - f0 + 1) % 16 == 0
+            assert all(l - f + 1 <= width for f, l in b)
+            assert len(b) == -(-rows // width)
+    g = np.random.default_rng(0)
+    T, E, k = 700, 12, 3
+    idx = np.stack([g.choice(E, k, replace=False) for _ in range(T)])
+    toks, tiles = schedule_cover_tokens(idx, E, 1, (32, 160))
+    for width in (32, 160):
+        n = 0
+        for e in range(E + 1):
+            rows = [t for t in range(T) if e == E or e in idx[t]]
+            for f, l in chunk_bounds(len(rows), width):
+                assert rows[f] in toks and rows[l] in toks
+                n += 1
+        assert tiles[width] == n

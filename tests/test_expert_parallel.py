@@ -1,8 +1,9 @@
 """Expert-parallel exchange logic (sparse_moe_layer_06_b200.expert_parallel) on
 two gloo ranks on CPU.  The per-rank compute steps (route, permute, grouped
 expert FFN, combine) are the oracle's, so the test checks exactly what the
-module adds: the row counts, the all-to-all splits, the regrouping by local
-expert and the inverse exchange.  Each rank's output must equal the oracle's
+module adds: the row counts, the block layout (each receiver gets its rows
+expert-major: local expert, then source rank), the point-to-point exchange of
+the blocks and the inverse exchange.  Each rank's output must equal the oracle's
 single-process layer on that rank's tokens with all experts."""
 import os
 import socket
@@ -120,3 +121,14 @@ def test_local_expert_range():
     assert local_expert_range(256, 3, 8) == (96, 32)
     with pytest.raises(ValueError):
         local_expert_range(10, 0, 4)
+
+
+def test_exchange_layout_expert_major():
+    from sparse_moe_layer_06_b200.expert_parallel import exchange_layout
+    send = [[2, 0, 1], [3, 4, 0]]          # to rank 0: experts 0..2; to rank 1: 0..2
+    recv = [[1, 5, 0], [2, 0, 7]]          # from rank 0 / rank 1 for my experts 0..2
+    send_off, recv_off, group_off = exchange_layout(send, recv)
+    assert send_off == [[0, 2, 2], [3, 6, 10]]          # destination-major, consecutive
+    # expert-major receive buffer: e0 (s0: 1, s1: 2), e1 (s0: 5, s1: 0), e2 (s0: 0, s1: 7)
+    assert recv_off == [[0, 3, 8], [1, 8, 8]]
+    assert group_off == [0, 3, 8, 15]

@@ -1,20 +1,23 @@
 """GPU parity at the five named workload configurations, in the launch
 configuration the benchmark times (moe_forward on the whole batch).
 
-Routing is compared with the oracle on every token; the layer output on a
-seeded sample of tokens (the oracle is per-token independent, so a sampled
-token is checked exactly as it would be in a full run)."""
+Routing is compared with the oracle on every token.  The layer output is
+compared on every token of the small batches and, at the large ones, on the
+tokens that cover every token tile of both expert GEMMs' schedules: the first
+and last row of every chunk of every expert segment and of the shared expert,
+derived from the GPU's own routing and the tile widths the launch used
+(moe_expert_tile_rows).  The oracle is per-token independent, so a checked
+token is checked exactly as in a full run."""
 import numpy as np
 import pytest
 import torch
 
-from parity_util import forward_parity, to_cpu_inputs
+from parity_util import forward_parity, schedule_cover_tokens, to_cpu_inputs
 from sparse_moe_layer_06_b200 import moe
 from sparse_moe_layer_06_b200.workloads import CONFIGS, make_inputs, make_x, sample_tokens
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
-N_SAMPLE = 24
 
 
 @pytest.fixture(scope="module")
@@ -42,11 +45,17 @@ def _run(c, inp):
     return out, idx, w
 
 
-def _check(c, inp, cpu, n_sample=N_SAMPLE):
+def _check(c, inp, cpu, all_tokens=False):
     out, idx, w = _run(c, inp)
     # routing on every token
     forward_parity_routing_only(inp, c, idx, w, cpu)
-    toks = sample_tokens(c.T, n_sample, seed=0)
+    if all_tokens:
+        toks = list(range(c.T))
+    else:
+        widths = moe.moe_expert_tile_rows(moe.MoEProblem.from_config(c))
+        toks, tiles = schedule_cover_tokens(idx.cpu().numpy(), c.E, c.num_shared, widths)
+        print(f"{c.name}: {len(toks)} tokens cover all tiles (tile widths {widths}: "
+              f"{tiles} tiles), coverage 1.0")
     n_ex, err, scale = forward_parity(inp, c, out, idx, w, tokens=toks, cpu_inp=cpu)
     return idx, n_ex, err, scale
 
@@ -64,7 +73,7 @@ def forward_parity_routing_only(inp, c, idx, w, cpu):
 def test_tiny_config():
     c = CONFIGS["tiny"]
     inp = make_inputs(c, seed=0, device=DEV)
-    _check(c, inp, to_cpu_inputs(inp), n_sample=c.T)
+    _check(c, inp, to_cpu_inputs(inp), all_tokens=True)
 
 
 def test_hy3_config():
@@ -85,7 +94,7 @@ def test_hy4_configs(name, hy4_weights):
         inp["logit_bias"] = skew_logit_bias(c.E).to(DEV)
     cpu = dict(wcpu, x=x.cpu(), logit_bias=None if inp["logit_bias"] is None
                else inp["logit_bias"].cpu())
-    idx, n_ex, err, scale = _check(c, inp, cpu, n_sample=c.T if c.T <= 64 else N_SAMPLE)
+    idx, n_ex, err, scale = _check(c, inp, cpu, all_tokens=c.T <= 64)
     counts = np.bincount(idx.cpu().numpy().ravel(), minlength=c.E)
     if name == "hy4_decode":
         assert 150 <= (counts > 0).sum() <= 256

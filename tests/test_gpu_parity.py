@@ -286,10 +286,14 @@ def test_forward_saturating_clamp():
 def test_forward_empty_batch_is_noop():
     c = cfg(T=0)
     p = moe.MoEProblem.from_config(c)
-    before = moe.moe_launch_count()
-    dummy = torch.zeros(16, dtype=c.dtype, device=DEV)
+    # T = 0 tokens, full-size weights: nothing is enqueued
+    inp = make_inputs(c.with_tokens(1), seed=1, device=DEV)
+    empty = torch.zeros(1, c.H, dtype=c.dtype, device=DEV)  # (a non-null pointer)
     ws = moe.alloc_workspace(p, moe.MOE_CALL_FORWARD)
-    moe.moe_forward(p, dummy, dummy, None, dummy, dummy, dummy, None, None, ws)
+    torch.cuda.synchronize()
+    before = moe.moe_launch_count()
+    moe.moe_forward(p, empty, inp["gate_w"], None, inp["expert_w"], inp["shared_w"], empty, None,
+                    None, ws)
     assert moe.moe_launch_count() == before
 
 
@@ -330,9 +334,11 @@ def test_forward_repeatable_and_staged_path_agrees():
 
 
 def test_forward_gather_variants_agree():
-    """The row gather inside the gate/up GEMM (MOE_FUSED_GATHER=1) and the
-    scatter-add combine (MOE_COMBINE=atomic) give the same layer: both are
-    checked against the oracle in a fresh process each."""
+    """The row gather inside the gate/up GEMM (MOE_FUSED_GATHER=1), the
+    scatter-add combine (MOE_COMBINE=atomic), the unrotated K order
+    (MOE_KROT=0) and ordinary launches without programmatic dependent launch
+    (MOE_PDL=0) give the same layer: each is checked against the oracle in a
+    fresh process."""
     import os
     import subprocess
     import sys
@@ -347,7 +353,8 @@ def test_forward_gather_variants_agree():
         "forward_parity(inp, c, out, idx, w); print('ok')")
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     for env in ({"MOE_FUSED_GATHER": "1"}, {"MOE_COMBINE": "atomic"},
-                {"MOE_FUSED_GATHER": "1", "MOE_COMBINE": "atomic"}):
+                {"MOE_FUSED_GATHER": "1", "MOE_COMBINE": "atomic"}, {"MOE_KROT": "0"},
+                {"MOE_PDL": "0"}, {"MOE_PDL": "0", "MOE_FUSED_GATHER": "1"}):
         r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True,
                            text=True, env={**os.environ, **env}, timeout=600)
         assert r.returncode == 0 and "ok" in r.stdout, (env, r.stdout[-2000:], r.stderr[-2000:])

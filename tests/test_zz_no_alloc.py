@@ -2,15 +2,16 @@
 device memory (for example code running during a CUDA stream capture, or a
 serving loop whose framework allocator owns all device memory).  It keeps its
 scratch in a fixed device array inside the library; this file checks it
-against moe_route, which takes a caller workspace, on two calls in a row with
-different inputs (so stale scratch from the first call would show up), and
-that a problem too large for the array is refused.  Collected last on
-purpose."""
+against moe_route, which takes a caller workspace, and against the CPU
+oracle's routing, on two calls in a row with different inputs (so stale
+scratch from the first call would show up), and that a problem too large for
+the array is refused.  Collected last on purpose."""
 import numpy as np
 import pytest
 import torch
 
-from parity_util import W_RTOL
+import oracle
+from parity_util import W_RTOL, check_routing, to_cpu_inputs
 from sparse_moe_layer_06_b200 import moe
 from sparse_moe_layer_06_b200.workloads import MoEConfig, make_inputs
 
@@ -35,6 +36,11 @@ def _route_both(c, seed, bias=None):
     w_b = torch.zeros(c.T, c.top_k, dtype=torch.float32, device=DEV)
     moe.moe_route_noalloc(p, inp["x"], inp["gate_w"], bias, idx_b, w_b)
     torch.cuda.synchronize()
+    # the no-allocation path against the oracle as well (near-ties validated)
+    cpu = to_cpu_inputs(inp)
+    orc = oracle.route(cpu["x"], cpu["gate_w"], c.top_k, c.routed_scale,
+                       logit_bias=None if bias is None else bias.cpu())
+    check_routing(idx_b.cpu().numpy(), w_b.cpu().numpy(), orc, c.top_k)
     return idx_a.cpu(), w_a.cpu(), idx_b.cpu(), w_b.cpu()
 
 
