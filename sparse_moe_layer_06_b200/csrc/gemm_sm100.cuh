@@ -159,19 +159,17 @@ struct GemmArgs {
     // still fixed), so CTAs running together read different K bands of the
     // weights instead of the same one in lockstep
     int32_t k_rotate;
-    // Programmatic dependent launch.  Before waiting for the grid it depends
-    // on, the producer pulls the first prefetch_ksteps weight steps of this
-    // CTA's first tile into L2 (weights never depend on an earlier launch);
-    // every thread that reads an earlier launch's output waits first.  With
+    // Programmatic dependent launch: every thread that reads an earlier
+    // launch's output waits for it first (griddepcontrol.wait).  With
     // pdl_trigger_early the next launch may start as soon as this grid has
-    // passed that wait (otherwise when each CTA finishes its tiles).
-    int32_t prefetch_ksteps;
+    // passed that wait (otherwise when each CTA has issued all its copies).
     int32_t pdl_trigger_early;
-    // Weight read-ahead: with each stage's copies the producer also pulls the
-    // weight box pf_dist steps further along the tile into L2, so more weight
-    // bytes are on their way from DRAM than the shared-memory ring holds
-    // (0 = off)
-    int32_t pf_dist;
+    // L2 policy of the weights of a segment cut into several token chunks:
+    // 0 evict-first (like a single-chunk segment), 1 normal, 2 evict-last.
+    // Every chunk of such a segment reads the same weight tiles, and the
+    // chunks run at about the same time, so keeping the tiles in L2 turns the
+    // later chunks' weight reads into L2 hits.
+    int32_t multi_chunk_policy;
 };
 
 // Compile-time shape of one instantiation.
@@ -435,32 +433,16 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
         // the special (shared-expert) segment's weights are re-read by every
         // token chunk of that segment: keep them in L2 rather than streaming
         const uint64_t pol_ws = pol_x;
+        // weights of a routed segment with several token chunks
+        const uint64_t pol_wm = !args.l2_hints                  ? ptx::policy_evict_normal()
+                                : args.multi_chunk_policy == 2 ? ptx::policy_evict_last()
+                                : args.multi_chunk_policy == 1 ? ptx::policy_evict_normal()
+                                                               : pol_w;
+        auto weight_policy = [&](const TileInfo& ti) -> uint64_t {
+            if (ti.special) return pol_ws;
+            return ss.prefix[ti.seg + 1] - ss.prefix[ti.seg] > 1 ? pol_wm : pol_w;
+        };
         const bf16_raw_ptr gsrc = reinterpret_cast<bf16_raw_ptr>(args.gather_src);
-        if (C::kSwiGLU || C::kDown) {
-            // weights of this CTA's first tile into L2 while the launch this
-            // one depends on may still be running (weights are never written)
-            if (lane == 0 && args.prefetch_ksteps > 0) {
-                for (int t = unit; t < total_tiles; t += units) {
-                    TileInfo ti;
-                    if (!decode(t, ti)) continue;
-                    const CUtensorMap* tA = ti.special ? &args.tmA1 : &args.tmA0;
-                    const int a_base = ti.special ? 0 : ti.seg * args.a_seg_stride;
-                    const uint64_t pw = ti.special ? pol_ws : pol_w;
-                    const int rot = k_rot(ti, ksteps);
-                    const int n = args.prefetch_ksteps < ksteps ? args.prefetch_ksteps : ksteps;
-                    for (int i = 0; i < n; ++i) {
-                        const int kb = i + rot < ksteps ? i + rot : i + rot - ksteps;
-                        const int k0 = kb * C::kKStep;
-                        if constexpr (C::kDown)
-                            ptx::tma_prefetch_3d(tA, 0, a_base + args.a_off0 + k0,
-                                                 ti.blk * (FP8 ? MB : 2 * MB), pw);
-                        else
-                            ptx::tma_prefetch_3d(tA, k0, ti.blk * 128, a_base + args.a_off0, pw);
-                    }
-                    break;
-                }
-            }
-        }
         // token rows (and, for a gathered tile, their indices) come from
         // earlier launches
         ptx::grid_dep_wait();
@@ -478,7 +460,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
             const CUtensorMap* tA = ti.special ? &args.tmA1 : &args.tmA0;
             const CUtensorMap* tB = ti.special ? args.tmB1 : args.tmB0;
             const int a_base = ti.special ? 0 : ti.seg * args.a_seg_stride;
-            const uint64_t pw = ti.special ? pol_ws : pol_w;
+            const uint64_t pw = weight_policy(ti);
             const bool gather =
                 C::kSwiGLU && !FP8 && !PAIR && args.gather_tok != nullptr && !ti.special;
             // GW > 0: the gather warps copy the rows; this warp only the weights
@@ -580,17 +562,6 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
                                 q += 16 << j;
                             }
                         }
-                    }
-                    if ((C::kSwiGLU || C::kDown) && args.pf_dist > 0 && i + args.pf_dist < span) {
-                        // read-ahead of a later weight box of this tile into L2
-                        const int ia = i + args.pf_dist;
-                        const int kp = kb_begin + (ia + rot < span ? ia + rot : ia + rot - span);
-                        const int kp0 = kp * C::kKStep;
-                        if constexpr (C::kDown)
-                            ptx::tma_prefetch_3d(tA, 0, a_base + args.a_off0 + kp0,
-                                                 ti.blk * (FP8 ? MB : 2 * MB), pw);
-                        else
-                            ptx::tma_prefetch_3d(tA, kp0, ti.blk * 128, a_base + args.a_off0, pw);
                     }
                 }
                 if (++stage == C::kStages) {

@@ -633,14 +633,19 @@ bool combine_atomic() {
     return v;
 }
 
-// MOE_FUSED_GATHER=1 makes the gate/up GEMM gather routed token rows straight
-// from x with cp.async (bf16 problems) instead of reading the permuted copy
-// x_perm.  Off by default: at prefill sizes the 16-byte copies throttle the
-// producer warp (measured 3x slower gate/up at 4096 tokens); at decode sizes
-// the two are even.
-bool fused_gather() {
-    const bool v = env_int("MOE_FUSED_GATHER", 0) != 0;
-    return v;
+// Whether the gate/up GEMM gathers the routed token rows straight from x
+// (four gather warps, 16-byte cp.async into the swizzled stage; bf16
+// problems) instead of reading a permuted copy x_perm written by a separate
+// gather kernel.  Default: fused for token tiles of up to 160 rows (measured
+// 0.2-2% faster per layer at the Hy4 prefill and decode and the Hy3 batches,
+// from dropping the gather launch and the copy's DRAM round trip), the
+// permuted copy for wider tiles (the 256-row tiles of the skewed batch, where
+// the gather warps slowed the tensor-bound GEMM by 10%).  MOE_FUSED_GATHER=0/1
+// forces either form.
+bool fused_gather(int nmax) {
+    const int v = env_int("MOE_FUSED_GATHER", -1);
+    if (v == 0 || v == 1) return v == 1;
+    return nmax <= 160;
 }
 
 // L2 cache hints on the GEMM operand loads (MOE_L2_HINTS=0 turns them off).
@@ -649,28 +654,22 @@ int l2_hints() {
     return v;
 }
 
-// Rotated K order in the expert GEMMs (MOE_KROT=0 turns it off): concurrent
-// tiles start their K loops at different offsets, spreading the weight reads
-// of the CTAs over the DRAM channels instead of sweeping one column band of
-// many rows in lockstep.
+// Rotated K order in the expert GEMMs (MOE_KROT=1; off by default):
+// concurrent tiles start their K loops at different offsets instead of
+// sweeping one column band of many rows in lockstep.  Measured 1.5% slower at
+// the Hy4 prefill batch and 4% slower at the skewed one (the DRAM channels
+// were already evenly loaded), so the plain order is the default.
 int k_rotate() {
-    const int v = env_int("MOE_KROT", 1) ? 1 : 0;
+    const int v = env_int("MOE_KROT", 0) ? 1 : 0;
     return v;
 }
 
 // Programmatic dependent launch along the forward's kernel chain (MOE_PDL=0
 // turns it off): each kernel may start while its predecessor finishes, does
-// its independent set-up (and, in the expert GEMMs, pulls its first weight
-// tiles into L2), then waits for the predecessor before reading its outputs.
+// its independent set-up (in the expert GEMMs: streams its first weight
+// tiles), then waits for the predecessor before reading its outputs.
 bool pdl_enabled() {
     const bool v = env_int("MOE_PDL", 1) != 0;
-    return v;
-}
-
-// Weight K-steps of each CTA's first tile prefetched into L2 before the
-// dependency wait of an expert GEMM launched programmatically (MOE_PREFETCH).
-int prefetch_ksteps() {
-    const int v = std::max(0, std::min(64, env_int("MOE_PREFETCH", 8)));
     return v;
 }
 
@@ -684,19 +683,23 @@ GemmArgs base_args(int32_t* status) {
     return a;
 }
 
-// Weight read-ahead distance of the expert GEMMs in pipeline steps
-// (MOE_PF_DIST; 0 = off).
-int pf_dist() {
-    const int v = std::max(0, std::min(32, env_int("MOE_PF_DIST", 0)));
-    return v;
+// L2 policy of the weights of an expert cut into several token chunks
+// (MOE_MULTI_CHUNK_L2: 0 evict-first, 1 normal (default), 2 evict-last).
+// With evict-first, the skewed batch's heavy experts had their weights
+// re-read from DRAM by almost every chunk (gate/up 29.4 GB of DRAM reads for
+// 9.8 GB of weights and token rows); evict-normal keeps them in L2 across the
+// chunks that run together (13.5 GB) and measured the fastest of the three.
+int multi_chunk_policy() {
+    const int v = env_int("MOE_MULTI_CHUNK_L2", 1);
+    return (v >= 0 && v <= 2) ? v : 1;
 }
 
-// Expert GEMM arguments for a launch that may start early (pdl): prefetch the
-// first weight tiles and let the following launch start early too.
-void expert_gemm_launch_args(GemmArgs& a, bool pdl, bool trigger_early) {
+// Expert GEMM arguments: K order, the multi-chunk weight policy, and whether
+// the following launch may start as soon as this one has passed its
+// dependency wait.
+void expert_gemm_launch_args(GemmArgs& a, bool trigger_early) {
     a.k_rotate = k_rotate();
-    a.pf_dist = pf_dist();
-    a.prefetch_ksteps = pdl ? prefetch_ksteps() : 0;
+    a.multi_chunk_policy = multi_chunk_policy();
     a.pdl_trigger_early = trigger_early ? 1 : 0;
 }
 
@@ -1129,7 +1132,7 @@ int32_t moe_grouped_swiglu_ffn(const moe_problem* p, const void* x_perm, int64_t
         a.clip = effective_clip(p);
         // an ordinary launch: the schedule it reads first is the previous
         // launch's output; the down GEMM may start as soon as it is resident
-        expert_gemm_launch_args(a, false, true);
+        expert_gemm_launch_args(a, true);
         MOE_TRY(launch_gemm<EPI_SWIGLU>(nmax, 2, a, max_tiles(rows, n_groups, nmax, I), s,
                                         "expert_gate_up_gemm"));
     }
@@ -1151,7 +1154,7 @@ int32_t moe_grouped_swiglu_ffn(const moe_problem* p, const void* x_perm, int64_t
         a.out_ld = static_cast<int32_t>(H);
         a.out_f32 = p->dtype == MOE_F32 ? 1 : 0;
         const bool pdl = pdl_enabled();
-        expert_gemm_launch_args(a, pdl, false);
+        expert_gemm_launch_args(a, false);
         MOE_TRY(launch_gemm<EPI_DOWN_STORE>(nmax, mb, a,
                                             max_tiles(rows, n_groups, nmax, H, 128 * mb), s,
                                             "expert_down_gemm", pdl));
@@ -1249,7 +1252,7 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
     const bool atomic_combine = combine_atomic();
     float* out_acc = atomic_combine ? at<float>(ws, L.out_acc) : nullptr;
     __nv_bfloat16* y_perm = at<__nv_bfloat16>(ws, L.y_perm);
-    const bool gather_in_gemm = !f32 && fused_gather();
+    const bool gather_in_gemm = !f32 && fused_gather(nmax);
     const void* x_b = x;
     if (f32) {
         MOE_TRY((run_gather<float, __nv_bfloat16>(static_cast<const float*>(x), T, p->H, p->top_k,
@@ -1299,7 +1302,7 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
         // (after a memset, the scatter-add mode's fused-gather form, the
         // launch is an ordinary one)
         const bool pdl_gu = pdl && !(gather_in_gemm && out_acc);
-        expert_gemm_launch_args(a, pdl_gu, true);
+        expert_gemm_launch_args(a, true);
         MOE_TRY(launch_gemm<EPI_SWIGLU>(nmax, 2, a, max_tiles(h_rows, nseg, nmax, I), s,
                                         "expert_gate_up_gemm", pdl_gu));
     }
@@ -1330,7 +1333,7 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
         a.row_weight = row_w;
         a.routed_rows = static_cast<int32_t>(T * k);
         const int64_t tiles = max_tiles(h_rows, nseg, nmax_dn, H, 128 * mb);
-        expert_gemm_launch_args(a, pdl, false);
+        expert_gemm_launch_args(a, false);
         if (atomic_combine) {
             a.out = out_acc;
             MOE_TRY(launch_gemm<EPI_DOWN_ATOMIC>(nmax_dn, mb, a, tiles, s,
@@ -1559,7 +1562,7 @@ int32_t moe_forward_fp8(const moe_problem* p, const void* x, const void* gate_w,
         a.scale_w_special = shared_s_gu;
         a.h_scale = h_scale;
         a.h_scale_inv = 1.0f / h_scale;
-        expert_gemm_launch_args(a, pdl, true);
+        expert_gemm_launch_args(a, true);
         MOE_TRY(launch_gemm_fp8<EPI_SWIGLU>(nmax, 2, a, max_tiles(h_rows, nseg, nmax, I), s,
                                             "expert_gate_up_gemm_fp8", pdl));
     }
@@ -1593,7 +1596,7 @@ int32_t moe_forward_fp8(const moe_problem* p, const void* x, const void* gate_w,
         a.scale_w_special = shared_s_d;
         a.h_scale = h_scale;
         a.h_scale_inv = 1.0f / h_scale;
-        expert_gemm_launch_args(a, pdl, false);
+        expert_gemm_launch_args(a, false);
         MOE_TRY(launch_gemm_fp8<EPI_DOWN_STORE>(nmax_dn, mb, a,
                                                 max_tiles(h_rows, nseg, nmax_dn, H, 128 * mb), s,
                                                 "expert_down_gemm_fp8", pdl));

@@ -134,18 +134,6 @@ __device__ __forceinline__ void tma_load_3d_pair(void* smem_dst, const CUtensorM
         : "memory");
 }
 
-// L2 prefetch of one 3D box of a tensor map (no shared memory, no barrier):
-// the lines are pulled into L2 so that a later tensor copy of the same box
-// hits there.  Same coordinate rules as a load.
-__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* m, int32_t c0, int32_t c1,
-                                                int32_t c2, uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.prefetch.tensor.3d.L2.global.tile.L2::cache_hint [%0, {%1, %2, %3}], "
-        "%4;" ::"l"(reinterpret_cast<uint64_t>(m)),
-        "r"(c0), "r"(c1), "r"(c2), "l"(policy)
-        : "memory");
-}
-
 // Programmatic dependent launch.  grid_dep_wait blocks the calling thread
 // until every grid this launch depends on has completed and its memory
 // operations are visible (it returns at once for a launch without such a

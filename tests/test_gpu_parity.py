@@ -334,11 +334,11 @@ def test_forward_repeatable_and_staged_path_agrees():
 
 
 def test_forward_gather_variants_agree():
-    """The row gather inside the gate/up GEMM (MOE_FUSED_GATHER=1), the
-    scatter-add combine (MOE_COMBINE=atomic), the unrotated K order
-    (MOE_KROT=0) and ordinary launches without programmatic dependent launch
-    (MOE_PDL=0) give the same layer: each is checked against the oracle in a
-    fresh process."""
+    """The permuted token copy instead of the row gather inside the gate/up
+    GEMM (MOE_FUSED_GATHER=0), the scatter-add combine (MOE_COMBINE=atomic),
+    the rotated K order (MOE_KROT=1), ordinary launches without programmatic
+    dependent launch (MOE_PDL=0) give the same layer: each is checked against
+    the oracle in a fresh process."""
     import os
     import subprocess
     import sys
@@ -352,9 +352,9 @@ def test_forward_gather_variants_agree():
         "out, idx, w = run_forward(c, inp);"
         "forward_parity(inp, c, out, idx, w); print('ok')")
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    for env in ({"MOE_FUSED_GATHER": "1"}, {"MOE_COMBINE": "atomic"},
-                {"MOE_FUSED_GATHER": "1", "MOE_COMBINE": "atomic"}, {"MOE_KROT": "0"},
-                {"MOE_PDL": "0"}, {"MOE_PDL": "0", "MOE_FUSED_GATHER": "1"}):
+    for env in ({"MOE_FUSED_GATHER": "0"}, {"MOE_COMBINE": "atomic"},
+                {"MOE_FUSED_GATHER": "0", "MOE_COMBINE": "atomic"}, {"MOE_KROT": "1"},
+                {"MOE_PDL": "0"}, {"MOE_PDL": "0", "MOE_FUSED_GATHER": "0"}):
         r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True,
                            text=True, env={**os.environ, **env}, timeout=600)
         assert r.returncode == 0 and "ok" in r.stdout, (env, r.stdout[-2000:], r.stderr[-2000:])
