@@ -461,6 +461,13 @@ def time_steps(step, n, stream, dist=None, device=None):
     return max_over_ranks(ev0.elapsed_time(ev1), dist, device) / n
 
 
+def cool_down(seconds):
+    """Let the GPU idle before the next pass, so that every pass starts from
+    the same state: a pass that follows seconds of full load would otherwise
+    run at the lower clock the 1 kW power limiter sets by then."""
+    time.sleep(max(0.5, seconds))
+
+
 def kernel_times(moe, step, n, device=None):
     """Per-kernel CUDA-event durations over n steps (the library records an
     event pair around each launch on its stream).  Those events also keep
@@ -490,7 +497,9 @@ def measure_workload(moe, cfg, inp, x, dev, stream, steps, warmup, fp8_weights=N
                         ws, stream)
     for _ in range(warmup):
         step()
+    cool_down(1.0)
     ms = time_steps(step, steps, stream, None, dev)
+    cool_down(2 * ms * steps / 1e3)
     kt = kernel_times(moe, step, steps, dev)
     status = moe.moe_read_device_status(ws)
     peaks, _ = read_peaks()
@@ -635,7 +644,9 @@ def main():
     launches = moe.moe_launch_count() - launches0
     clock_rec = clocks.summary(wall1 - ms_per_step * args.steps / 1e3, wall1)
     # per-kernel durations: the same number of steps again, with an event pair
-    # around every launch (a separate pass: the events keep launches apart)
+    # around every launch (a separate pass: the events keep launches apart),
+    # after an idle pause as long as the timed region ran, twice over
+    cool_down(2 * ms_per_step * args.steps / 1e3)
     kt = kernel_times(moe, step, args.steps, dev)
     if dist:
         dist.barrier()
@@ -678,6 +689,7 @@ def main():
 
     e2e_steps(3)
     torch.cuda.synchronize(dev)
+    cool_down(2 * ms_per_step * args.e2e_steps / 1e3)
     if dist:
         dist.barrier()
     e0 = torch.cuda.Event(enable_timing=True)

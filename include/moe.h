@@ -35,7 +35,9 @@
  *  - Errors are returned, never thrown; on any error nothing is enqueued.
  *  - dtype: MOE_BF16 - x, weights, outputs bf16; all sums in fp32 on tensor
  *    cores.  MOE_F32 - x, weights, outputs fp32; the router runs in fp32 on
- *    CUDA cores, the expert GEMMs run on bf16 copies made on the device.
+ *    CUDA cores, the expert GEMMs on tensor cores reading the fp32 operands
+ *    as TF32 (10-bit mantissa; tcgen05 kind::tf32), with fp32 sums, and h and
+ *    the expert output rows stay fp32.
  *  - Shapes supported: T >= 0 (T == 0 is a no-op), H and I multiples of 64,
  *    1 <= top_k <= min(E, 32), E <= 256, num_shared in {0,1},
  *    T*top_k < 2^31.  Anything else returns MOE_ERR_UNSUPPORTED.

@@ -178,9 +178,11 @@ struct GemmArgs {
 //         EPI_SWIGLU (MB = 2), else 1 or 2 adjacent 128-row blocks of one
 //         matrix (two MMAs sharing each token tile)
 // The pipeline depth is whatever fits the 227 KB of shared memory.
-//   FP8   E4M3 operands (kind::f8f6f4): 128 K-elements per 128-byte row per
-//         stage instead of 64, scales applied in the epilogue
-template <int EPI, int NMAX, int MB, bool FP8 = false, bool PAIR = false, int GW = 0>
+//   ET    operand element type: 0 bf16 (kind::f16), 1 E4M3 (kind::f8f6f4:
+//         128 K-elements per 128-byte row per stage instead of 64, scales
+//         applied in the epilogue), 2 fp32 read as TF32 (kind::tf32: 32
+//         K-elements per 128-byte row; h and the output rows stay fp32)
+template <int EPI, int NMAX, int MB, int ET = 0, bool PAIR = false, int GW = 0>
 struct GemmCfg {
     static_assert(NMAX % 16 == 0 && NMAX >= 16 && NMAX <= 256, "N tile");
     static_assert(MB == 1 || MB == 2, "weight sub-tiles");
@@ -188,7 +190,11 @@ struct GemmCfg {
     static constexpr bool kSwiGLU = (EPI == EPI_SWIGLU);
     static constexpr bool kDown = (EPI == EPI_DOWN_ATOMIC || EPI == EPI_DOWN_STORE);
     static constexpr int kNumA = MB;
-    static constexpr int kKStep = FP8 ? 128 : 64;  // K elements per stage (128-byte rows)
+    static_assert(ET >= 0 && ET <= 2, "element type");
+    static constexpr bool kFP8 = (ET == 1);
+    static constexpr bool kTF32 = (ET == 2);
+    static constexpr int kElemBytes = kFP8 ? 1 : (kTF32 ? 4 : 2);
+    static constexpr int kKStep = 128 / kElemBytes;  // K elements per stage (128-byte rows)
     static constexpr int kATileBytes = 128 * 128;  // 128 rows x 64 bf16
     static constexpr int kABytes = kNumA * kATileBytes;
     // PAIR: the two CTAs of a cluster run one tile with cta_group::2 MMAs of
@@ -213,7 +219,7 @@ struct GemmCfg {
     static constexpr int kBarrierBytes = 512;
     // (rounded to 128 bytes so that what follows stays 128-byte aligned)
     static constexpr int kSchedBytes = (5 * (kMaxSegments + 1) * 4 + 127) / 128 * 128;
-    static constexpr bool kMeta = kDown || (kSwiGLU && FP8);  // per-column metadata
+    static constexpr bool kMeta = kDown || (kSwiGLU && kFP8);  // per-column metadata
     static constexpr int kMetaBytes = kMeta ? 2 * NMAX * 8 : 0;
     static constexpr int kEpiWarps = 8;
     // EPI_SWIGLU: token index of each row of the current tile (row gather)
@@ -230,7 +236,7 @@ struct GemmCfg {
     static_assert((2 * kStages + 7) * 8 + 3 * 4 <= kBarrierBytes, "barrier area");
     // GW > 0 (EPI_SWIGLU with the row gather): that many more warps copy the
     // gathered token rows; the producer warp then only issues the weight copies
-    static_assert(GW == 0 || (EPI == EPI_SWIGLU && !FP8 && !PAIR), "gather warps");
+    static_assert(GW == 0 || (EPI == EPI_SWIGLU && ET == 0 && !PAIR), "gather warps");
     static constexpr int kThreads = 32 * (2 + kEpiWarps + GW);
 };
 
@@ -297,10 +303,12 @@ __device__ __forceinline__ float clamp_keep_nan(float v, float lim) {
     return v > lim ? lim : (v < -lim ? -lim : v);
 }
 
-template <int EPI, int NMAX, int MB, bool FP8, bool PAIR, int GW>
-__global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThreads, 1)
+template <int EPI, int NMAX, int MB, int ET, bool PAIR, int GW>
+__global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, ET, PAIR, GW>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmArgs args) {
-    using C = GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>;
+    using C = GemmCfg<EPI, NMAX, MB, ET, PAIR, GW>;
+    constexpr bool FP8 = C::kFP8;
+    constexpr bool TF32 = C::kTF32;
     constexpr int CG = PAIR ? 2 : 1;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned ring (the 128-byte swizzle atoms need it)
@@ -462,7 +470,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
             const int a_base = ti.special ? 0 : ti.seg * args.a_seg_stride;
             const uint64_t pw = weight_policy(ti);
             const bool gather =
-                C::kSwiGLU && !FP8 && !PAIR && args.gather_tok != nullptr && !ti.special;
+                C::kSwiGLU && ET == 0 && !PAIR && args.gather_tok != nullptr && !ti.special;
             // GW > 0: the gather warps copy the rows; this warp only the weights
             const bool own_gather = gather && GW == 0;
             // token rows this CTA loads (PAIR: its half of the tile's columns)
@@ -541,8 +549,9 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
                     if constexpr (C::kDown) {
                         // MN-major A: one 3D copy of the tile's 128-byte-wide H
                         // chunks (bf16: 2*MB chunks of 64 values x 64 K-rows;
-                        // FP8: MB chunks of 128 values x 128 K-rows), chunk-major
-                        load3d(sA, tA, 0, a_base + args.a_off0 + k0, ti.blk * (FP8 ? MB : 2 * MB),
+                        // FP8: MB chunks of 128 values x 128 K-rows; TF32:
+                        // 4*MB chunks of 32 values x 32 K-rows), chunk-major
+                        load3d(sA, tA, 0, a_base + args.a_off0 + k0, ti.blk * (C::kElemBytes * MB),
                                pw);
                     } else if constexpr (C::kSwiGLU) {
                         // gate and up tiles (adjacent matrices) in one 3D copy
@@ -589,11 +598,14 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
             uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
             bool ok = true;
             constexpr uint32_t kAMajor = C::kDown ? 1u : 0u;
-            // MN-major A: per MMA (K = 16 bf16 / 32 FP8) the next 16 / 32 K-rows
-            // of 128 bytes; between 128-byte H chunks 8 KB (bf16: two chunks per
-            // 128-row sub-tile) -- unused for FP8, where one chunk is 128 rows
-            constexpr uint32_t kMnStep = FP8 ? 4096u : 2048u;
-            constexpr uint32_t kMnLbo = FP8 ? 16384u : 8192u;
+            // MN-major A: per MMA (32 bytes of K: 16 bf16 / 32 FP8 / 8 TF32)
+            // the next 16 / 32 / 8 K-rows of 128 bytes; between 128-byte H
+            // chunks one stage's K-rows: 8 KB (bf16: two chunks per 128-row
+            // sub-tile), 4 KB (TF32: four chunks) -- unused for FP8, where one
+            // chunk is the 128 rows.  TF32 tiles use the 128-byte swizzle with
+            // 32-byte atoms (the copies write it; see make_tmap_down)
+            constexpr uint32_t kMnStep = 4096u / C::kElemBytes;
+            constexpr uint32_t kMnLbo = 16384u / C::kElemBytes;
             // PAIR: arrive on the barrier at the same offset in both CTAs
             auto commit = [&](uint64_t* bar) {
                 if constexpr (PAIR) {
@@ -616,8 +628,9 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
                 }
                 ptx::tc_fence_after();
                 const uint32_t d0 = tmem_base + acc * C::kAccCols;
-                const uint32_t idesc = FP8 ? ptx::idesc_e4m3_f32(kM, ti.n_mma, kAMajor, 0)
-                                           : ptx::idesc_bf16_f32(kM, ti.n_mma, kAMajor, 0);
+                const uint32_t idesc = FP8    ? ptx::idesc_e4m3_f32(kM, ti.n_mma, kAMajor, 0)
+                                       : TF32 ? ptx::idesc_tf32_f32(kM, ti.n_mma, kAMajor, 0)
+                                              : ptx::idesc_bf16_f32(kM, ti.n_mma, kAMajor, 0);
                 for (int i = 0; i < span; ++i) {
                     if (!ptx::mbar_wait(&full_bar[stage], phase, abort_flag)) {
                         fail(DEV_ERR_TIMEOUT);
@@ -637,11 +650,15 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
 #pragma unroll
                         for (int j = 0; j < MB; ++j) {
                             const uint32_t a_sub = a_addr + j * C::kATileBytes;
+                            // (TF32 MN-major: the 32-byte-atom swizzle, 4-row K groups)
                             const uint64_t adesc =
-                                C::kDown ? ptx::smem_desc_sw128(a_sub + kk * kMnStep, kMnLbo, 1024)
-                                         : ptx::smem_desc_sw128(a_sub + kk * 32, 16, 1024);
+                                !C::kDown ? ptx::smem_desc_sw128(a_sub + kk * 32, 16, 1024)
+                                : TF32    ? ptx::smem_desc_sw128_32b(a_sub + kk * kMnStep, kMnLbo, 512)
+                                          : ptx::smem_desc_sw128(a_sub + kk * kMnStep, kMnLbo, 1024);
                             if constexpr (FP8)
                                 ptx::mma_fp8<CG>(d0 + j * NMAX, adesc, bdesc, idesc, accum);
+                            else if constexpr (TF32)
+                                ptx::mma_tf32<CG>(d0 + j * NMAX, adesc, bdesc, idesc, accum);
                             else
                                 ptx::mma_bf16<CG>(d0 + j * NMAX, adesc, bdesc, idesc, accum);
                         }
@@ -824,6 +841,18 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>::kThread
                         // reciprocal (both ~1e-7 relative, far below bf16)
                         hv[j] = gg * fast_rcp(1.0f + __expf(-gg)) * uu;
                         if constexpr (FP8) hv[j] *= args.h_scale_inv;  // exact: power of two
+                    }
+                    if constexpr (TF32) {
+                        // fp32 h: each lane stores its own row's value; the 32
+                        // lanes of a column write 128 consecutive bytes
+                        float* hf = reinterpret_cast<float*>(args.out);
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            if (m_ok && c0 + j < ti.n_valid)
+                                hf[static_cast<size_t>(ti.out_row + c0 + j) * args.out_ld + m] =
+                                    hv[j];
+                        }
+                        return;
                     }
 #pragma unroll
                     for (int j = 0; j < 16; j += 2) {

@@ -110,6 +110,7 @@ struct ElemType {
 };
 constexpr ElemType kBF16{CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2};
 constexpr ElemType kU8{CU_TENSOR_MAP_DATA_TYPE_UINT8, 1};
+constexpr ElemType kF32{CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4};
 
 int env_int(const char* name, int dflt);
 
@@ -162,10 +163,11 @@ bool make_tmap_gateup(CUtensorMap* m, const void* ptr, int64_t n_mats, int64_t I
     return r == CUDA_SUCCESS;
 }
 
-// Down-projection weights [rows, H] (H contiguous) as a 3D tensor {64, rows,
-// H/64}: dim 0 = 64 consecutive H values, dim 1 = the row (stride H*2 bytes),
-// dim 2 = which 64-wide H chunk (stride 128 bytes).  A {64, 64, 2*mb} box is
-// one K-step of 2*mb chunks, laid out chunk by chunk in shared memory.
+// Down-projection weights [rows, H] (H contiguous) as a 3D tensor {c, rows,
+// H/c} with c = 128 bytes of H values (64 bf16, 128 E4M3, 32 fp32): dim 0 = c
+// consecutive H values, dim 1 = the row, dim 2 = which c-wide H chunk (stride
+// 128 bytes).  A {c, c, bytes*mb} box is one K-step of the chunks of mb
+// 128-row sub-tiles, laid out chunk by chunk in shared memory.
 bool make_tmap_down(CUtensorMap* m, const void* ptr, int64_t rows, int64_t H, int mb,
                     ElemType et = kBF16) {
     EncodeTiledFn fn = encode_fn();
@@ -176,10 +178,14 @@ bool make_tmap_down(CUtensorMap* m, const void* ptr, int64_t rows, int64_t H, in
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(H) * et.bytes, 128u};
     // one K-step: 64 (bf16) or 128 (FP8) rows of each of the tile's chunks
     cuuint32_t box[3] = {static_cast<cuuint32_t>(chunk), static_cast<cuuint32_t>(chunk),
-                         static_cast<cuuint32_t>(et.bytes == 2 ? 2 * mb : mb)};
+                         static_cast<cuuint32_t>(et.bytes * mb)};
     cuuint32_t estr[3] = {1u, 1u, 1u};
+    // fp32 (TF32) MN-major operands take the 128-byte swizzle with 32-byte
+    // atoms, the only MN-major shared-memory layout TF32 MMAs accept
+    const CUtensorMapSwizzle sw =
+        et.bytes == 4 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B;
     CUresult r = fn(m, et.dt, 3, const_cast<void*>(ptr), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                     weight_l2_promotion(), CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -319,7 +325,7 @@ struct Carve {
 struct Layout {
     size_t status, logits, rcount, idx, w, hist, base, counts, offsets, partial, sched_gu, sched_dn,
         pos, src, row_w;
-    size_t x_perm, x_bf16, w_bf16, ws_bf16, h_perm, out_acc, y_perm, x_q, s_x, total;
+    size_t x_perm, h_perm, out_acc, y_perm, x_q, s_x, total;
 };
 
 int64_t perm_chunks(int64_t T) { return (T + kPermTokens - 1) / kPermTokens; }
@@ -346,11 +352,8 @@ Layout layout_for(const moe_problem* p, int call, int64_t ffn_rows = 0, int ffn_
         case MOE_CALL_FFN:
             L.sched_gu = c.take(sched_bytes());
             L.sched_dn = c.take(sched_bytes());
-            L.h_perm = c.take(ffn_rows * I * 2);
-            if (f32) {
-                L.x_bf16 = c.take(ffn_rows * H * 2);
-                L.w_bf16 = c.take(static_cast<int64_t>(ffn_groups) * 3 * I * H * 2);
-            }
+            // fp32 problems keep h in fp32 (TF32 operand of the down GEMM)
+            L.h_perm = c.take(ffn_rows * I * (f32 ? 4 : 2));
             break;
         case MOE_CALL_COMBINE:
             break;
@@ -397,17 +400,14 @@ Layout layout_for(const moe_problem* p, int call, int64_t ffn_rows = 0, int ffn_
             L.pos = c.take(T * k * 4);
             L.src = c.take(T * k * 4);
             L.row_w = c.take(T * k * 4);
-            L.x_perm = c.take(T * k * H * 2);
-            L.h_perm = c.take(T * (k + S) * I * 2);
+            // (fp32 problems: the permuted rows, h and the weighted rows in
+            // fp32, the operands and results of the TF32 GEMMs)
+            L.x_perm = c.take(T * k * H * (f32 ? 4 : 2));
+            L.h_perm = c.take(T * (k + S) * I * (f32 ? 4 : 2));
             // weighted expert rows (gather combine) or the fp32 token
             // accumulator (scatter-add combine) share one region
-            L.out_acc = c.take(std::max(T * (k + S) * H * 2, T * H * 4));
+            L.out_acc = c.take(std::max(T * (k + S) * H * (f32 ? 4 : 2), T * H * 4));
             L.y_perm = L.out_acc;
-            if (f32) {
-                L.x_bf16 = c.take(T * H * 2);
-                L.w_bf16 = c.take(E * 3 * I * H * 2);
-                L.ws_bf16 = c.take(S * 3 * I * H * 2);
-            }
             break;
     }
     L.total = c.off;
@@ -465,11 +465,11 @@ int resident_pairs(K kern, int threads, int smem) {
     return n;
 }
 
-template <int EPI, int NMAX, int MB, bool FP8 = false, bool PAIR = false, int GW = 0>
+template <int EPI, int NMAX, int MB, int ET = 0, bool PAIR = false, int GW = 0>
 int32_t launch_gemm_n(const GemmArgs& a, int grid, cudaStream_t s, const char* name,
                       bool coop = false, bool pdl = false) {
-    using C = GemmCfg<EPI, NMAX, MB, FP8, PAIR, GW>;
-    auto kern = grouped_gemm_kernel<EPI, NMAX, MB, FP8, PAIR, GW>;
+    using C = GemmCfg<EPI, NMAX, MB, ET, PAIR, GW>;
+    auto kern = grouped_gemm_kernel<EPI, NMAX, MB, ET, PAIR, GW>;
     int dev = 0;
     cudaGetDevice(&dev);
     static std::atomic<uint64_t> configured{0};
@@ -537,24 +537,24 @@ bool use_pair() {
     return v;
 }
 
-template <int EPI, int MB, bool FP8 = false>
+template <int EPI, int MB, int ET = 0>
 int32_t launch_gemm_mb(int nmax, const GemmArgs& a, int grid, cudaStream_t s, const char* name,
                        bool pair = false, bool pdl = false) {
     switch (nmax) {
-        case 16: return launch_gemm_n<EPI, 16, MB, FP8>(a, grid, s, name, false, pdl);
-        case 32: return launch_gemm_n<EPI, 32, MB, FP8>(a, grid, s, name, false, pdl);
+        case 16: return launch_gemm_n<EPI, 16, MB, ET>(a, grid, s, name, false, pdl);
+        case 32: return launch_gemm_n<EPI, 32, MB, ET>(a, grid, s, name, false, pdl);
         case 64:
-            return pair ? launch_gemm_n<EPI, 64, MB, FP8, true>(a, grid, s, name, false, pdl)
-                        : launch_gemm_n<EPI, 64, MB, FP8>(a, grid, s, name, false, pdl);
+            return pair ? launch_gemm_n<EPI, 64, MB, ET, true>(a, grid, s, name, false, pdl)
+                        : launch_gemm_n<EPI, 64, MB, ET>(a, grid, s, name, false, pdl);
         case 128:
-            return pair ? launch_gemm_n<EPI, 128, MB, FP8, true>(a, grid, s, name, false, pdl)
-                        : launch_gemm_n<EPI, 128, MB, FP8>(a, grid, s, name, false, pdl);
+            return pair ? launch_gemm_n<EPI, 128, MB, ET, true>(a, grid, s, name, false, pdl)
+                        : launch_gemm_n<EPI, 128, MB, ET>(a, grid, s, name, false, pdl);
         case 160:
-            return pair ? launch_gemm_n<EPI, 160, MB, FP8, true>(a, grid, s, name, false, pdl)
-                        : launch_gemm_n<EPI, 160, MB, FP8>(a, grid, s, name, false, pdl);
+            return pair ? launch_gemm_n<EPI, 160, MB, ET, true>(a, grid, s, name, false, pdl)
+                        : launch_gemm_n<EPI, 160, MB, ET>(a, grid, s, name, false, pdl);
         case 256:
-            return pair ? launch_gemm_n<EPI, 256, MB, FP8, true>(a, grid, s, name, false, pdl)
-                        : launch_gemm_n<EPI, 256, MB, FP8>(a, grid, s, name, false, pdl);
+            return pair ? launch_gemm_n<EPI, 256, MB, ET, true>(a, grid, s, name, false, pdl)
+                        : launch_gemm_n<EPI, 256, MB, ET>(a, grid, s, name, false, pdl);
         default: return MOE_ERR_UNSUPPORTED;
     }
 }
@@ -566,11 +566,25 @@ int32_t launch_gemm_fp8(int nmax, int mb, const GemmArgs& a, int64_t max_tiles, 
     int grid = static_cast<int>(std::min<int64_t>(sm_count(), std::max<int64_t>(1, max_tiles)));
     const bool pair = use_pair() && nmax >= 64;
     if constexpr (EPI == EPI_SWIGLU) {
-        return launch_gemm_mb<EPI, 2, true>(nmax, a, grid, s, name, pair, pdl);
+        return launch_gemm_mb<EPI, 2, 1>(nmax, a, grid, s, name, pair, pdl);
     } else {
         static_assert(EPI == EPI_DOWN_STORE, "FP8 down GEMM uses the store epilogue");
-        if (mb == 2) return launch_gemm_mb<EPI, 2, true>(nmax, a, grid, s, name, pair, pdl);
-        return launch_gemm_mb<EPI, 1, true>(nmax, a, grid, s, name, false, pdl);
+        if (mb == 2) return launch_gemm_mb<EPI, 2, 1>(nmax, a, grid, s, name, pair, pdl);
+        return launch_gemm_mb<EPI, 1, 1>(nmax, a, grid, s, name, false, pdl);
+    }
+}
+
+// TF32 expert GEMMs on fp32 operands (fp32 problems): gate/up (+SwiGLU, fp32
+// h) and down (store or scatter-add epilogue), one CTA per tile.
+template <int EPI>
+int32_t launch_gemm_tf32(int nmax, int mb, const GemmArgs& a, int64_t max_tiles, cudaStream_t s,
+                         const char* name, bool pdl = false) {
+    int grid = static_cast<int>(std::min<int64_t>(sm_count(), std::max<int64_t>(1, max_tiles)));
+    if constexpr (EPI == EPI_SWIGLU) {
+        return launch_gemm_mb<EPI, 2, 2>(nmax, a, grid, s, name, false, pdl);
+    } else {
+        if (mb == 2) return launch_gemm_mb<EPI, 2, 2>(nmax, a, grid, s, name, false, pdl);
+        return launch_gemm_mb<EPI, 1, 2>(nmax, a, grid, s, name, false, pdl);
     }
 }
 
@@ -583,12 +597,12 @@ int32_t launch_gemm(int nmax, int mb, const GemmArgs& a, int64_t max_tiles, cuda
         if (a.gather_tok != nullptr) {
             // row gather by four dedicated gather warps
             switch (nmax) {
-                case 16: return launch_gemm_n<EPI, 16, 2, false, false, 4>(a, grid, s, name, false, pdl);
-                case 32: return launch_gemm_n<EPI, 32, 2, false, false, 4>(a, grid, s, name, false, pdl);
-                case 64: return launch_gemm_n<EPI, 64, 2, false, false, 4>(a, grid, s, name, false, pdl);
-                case 128: return launch_gemm_n<EPI, 128, 2, false, false, 4>(a, grid, s, name, false, pdl);
-                case 160: return launch_gemm_n<EPI, 160, 2, false, false, 4>(a, grid, s, name, false, pdl);
-                case 256: return launch_gemm_n<EPI, 256, 2, false, false, 4>(a, grid, s, name, false, pdl);
+                case 16: return launch_gemm_n<EPI, 16, 2, 0, false, 4>(a, grid, s, name, false, pdl);
+                case 32: return launch_gemm_n<EPI, 32, 2, 0, false, 4>(a, grid, s, name, false, pdl);
+                case 64: return launch_gemm_n<EPI, 64, 2, 0, false, 4>(a, grid, s, name, false, pdl);
+                case 128: return launch_gemm_n<EPI, 128, 2, 0, false, 4>(a, grid, s, name, false, pdl);
+                case 160: return launch_gemm_n<EPI, 160, 2, 0, false, 4>(a, grid, s, name, false, pdl);
+                case 256: return launch_gemm_n<EPI, 256, 2, 0, false, 4>(a, grid, s, name, false, pdl);
                 default: return MOE_ERR_UNSUPPORTED;
             }
         }
@@ -818,14 +832,6 @@ int32_t run_route(const moe_problem* p, const void* x, const void* gate_w, const
     return run_topk(p, logits, bias, idx, w, s, lp.splits, keep_sum);
 }
 
-int32_t run_cast(const void* in, void* out, int64_t n, cudaStream_t s) {
-    const int64_t blocks = std::min<int64_t>((n + 255) / 256, 148 * 16);
-    MOE_LAUNCH("cast_f32_bf16", s,
-               cast_f32_bf16_kernel<<<static_cast<unsigned>(std::max<int64_t>(1, blocks)), 256, 0,
-                                      s>>>(static_cast<const float*>(in),
-                                           static_cast<__nv_bfloat16*>(out), n));
-    return MOE_OK;
-}
 
 template <typename TIn, typename TOut>
 int32_t run_gather(const TIn* x, int64_t T, int H, int k, const int32_t* pos, int64_t n_rows,
@@ -928,18 +934,19 @@ int32_t run_gather(const TIn* x, int64_t T, int H, int k, const int32_t* pos, in
 
 // out[t] = sum over the token's rows of y (slot order, the shared row last),
 // one warp per (token, segment of H).
-template <typename TOut>
-int32_t run_gather_sum(const __nv_bfloat16* y, const int32_t* pos, int64_t T, int H, int k,
+template <typename TIn, typename TOut>
+int32_t run_gather_sum(const TIn* y, const int32_t* pos, int64_t T, int H, int k,
                        int64_t n_rows, int64_t shared_row0, TOut* out, int32_t* status,
                        cudaStream_t s, bool pdl = false) {
     const int warps = 8;
-    const int64_t segs = (H / 8 + kSegVecs - 1) / kSegVecs;
+    const int vec = 16 / static_cast<int>(sizeof(TIn));
+    const int64_t segs = (H / vec + kSegVecs - 1) / kSegVecs;
     const int blocks = static_cast<int>((T * segs + warps - 1) / warps);
     // two rows' loads in flight per lane before adding: measured faster than
     // wider batches, whose register use lowers the number of resident warps
     MOE_LAUNCH("combine_gather", s,
-               if (launch_ex(gather_sum_kernel<TOut, 2>, blocks, warps * 32, 0, s, pdl, y, pos, T,
-                             H, k, n_rows, shared_row0, out, status) != cudaSuccess)
+               if (launch_ex(gather_sum_kernel<TIn, TOut, 2>, blocks, warps * 32, 0, s, pdl, y,
+                             pos, T, H, k, n_rows, shared_row0, out, status) != cudaSuccess)
                    return MOE_ERR_CUDA);
     return MOE_OK;
 }
@@ -1101,24 +1108,21 @@ int32_t moe_grouped_swiglu_ffn(const moe_problem* p, const void* x_perm, int64_t
     const int64_t H = p->H, I = p->I;
     const void* xb = x_perm;
     const void* wb = expert_w;
-    if (p->dtype == MOE_F32) {
-        MOE_TRY(run_cast(x_perm, at<void>(ws, L.x_bf16), rows * H, s));
-        MOE_TRY(run_cast(expert_w, at<void>(ws, L.w_bf16), n_groups * 3 * I * H, s));
-        xb = at<void>(ws, L.x_bf16);
-        wb = at<void>(ws, L.w_bf16);
-    }
+    // fp32 problems: TF32 GEMMs on the fp32 operands as given
+    const bool f32 = p->dtype == MOE_F32;
+    const ElemType et = f32 ? kF32 : kBF16;
     const int nmax = pick_nmax(static_cast<double>(rows) / n_groups);
     int32_t* sg = at<int32_t>(ws, L.sched_gu);
     int32_t* sd = at<int32_t>(ws, L.sched_dn);
     MOE_LAUNCH("ffn_schedule", s,
                schedule_from_offsets_kernel<<<1, 32, 0, s>>>(offsets, n_groups, rows, sg, nmax, sd,
                                                              nmax, status));
-    __nv_bfloat16* h = at<__nv_bfloat16>(ws, L.h_perm);
+    void* h = at<void>(ws, L.h_perm);
     {
         GemmArgs a = base_args(status);
-        if (!make_tmap_gateup(&a.tmA0, wb, static_cast<int64_t>(n_groups) * 3, I, H))
+        if (!make_tmap_gateup(&a.tmA0, wb, static_cast<int64_t>(n_groups) * 3, I, H, et))
             return MOE_ERR_CUDA;
-        if (!make_tmap_rows(a.tmB0, xb, rows, H)) return MOE_ERR_CUDA;
+        if (!make_tmap_rows(a.tmB0, xb, rows, H, et)) return MOE_ERR_CUDA;
         a.tmA1 = a.tmA0;
         for (int j = 0; j < kNumBoxSizes; ++j) a.tmB1[j] = a.tmB0[j];
         a.sched = sg;
@@ -1133,15 +1137,19 @@ int32_t moe_grouped_swiglu_ffn(const moe_problem* p, const void* x_perm, int64_t
         // an ordinary launch: the schedule it reads first is the previous
         // launch's output; the down GEMM may start as soon as it is resident
         expert_gemm_launch_args(a, true);
-        MOE_TRY(launch_gemm<EPI_SWIGLU>(nmax, 2, a, max_tiles(rows, n_groups, nmax, I), s,
-                                        "expert_gate_up_gemm"));
+        if (f32)
+            MOE_TRY(launch_gemm_tf32<EPI_SWIGLU>(nmax, 2, a, max_tiles(rows, n_groups, nmax, I), s,
+                                                 "expert_gate_up_gemm_tf32"));
+        else
+            MOE_TRY(launch_gemm<EPI_SWIGLU>(nmax, 2, a, max_tiles(rows, n_groups, nmax, I), s,
+                                            "expert_gate_up_gemm"));
     }
     {
         GemmArgs a = base_args(status);
         const int mb = pick_down_mb(nmax);
-        if (!make_tmap_down(&a.tmA0, wb, static_cast<int64_t>(n_groups) * 3 * I, H, mb))
+        if (!make_tmap_down(&a.tmA0, wb, static_cast<int64_t>(n_groups) * 3 * I, H, mb, et))
             return MOE_ERR_CUDA;
-        if (!make_tmap_rows(a.tmB0, h, rows, I)) return MOE_ERR_CUDA;
+        if (!make_tmap_rows(a.tmB0, h, rows, I, et)) return MOE_ERR_CUDA;
         a.tmA1 = a.tmA0;
         for (int j = 0; j < kNumBoxSizes; ++j) a.tmB1[j] = a.tmB0[j];
         a.sched = sd;
@@ -1152,12 +1160,17 @@ int32_t moe_grouped_swiglu_ffn(const moe_problem* p, const void* x_perm, int64_t
         a.a_off0 = static_cast<int32_t>(2 * I);
         a.out = y_perm;
         a.out_ld = static_cast<int32_t>(H);
-        a.out_f32 = p->dtype == MOE_F32 ? 1 : 0;
+        a.out_f32 = f32 ? 1 : 0;
         const bool pdl = pdl_enabled();
         expert_gemm_launch_args(a, false);
-        MOE_TRY(launch_gemm<EPI_DOWN_STORE>(nmax, mb, a,
-                                            max_tiles(rows, n_groups, nmax, H, 128 * mb), s,
-                                            "expert_down_gemm", pdl));
+        if (f32)
+            MOE_TRY(launch_gemm_tf32<EPI_DOWN_STORE>(nmax, mb, a,
+                                                     max_tiles(rows, n_groups, nmax, H, 128 * mb),
+                                                     s, "expert_down_gemm_tf32", pdl));
+        else
+            MOE_TRY(launch_gemm<EPI_DOWN_STORE>(nmax, mb, a,
+                                                max_tiles(rows, n_groups, nmax, H, 128 * mb), s,
+                                                "expert_down_gemm", pdl));
     }
     return MOE_OK;
 }
@@ -1213,17 +1226,11 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
     float* w = w_out ? w_out : at<float>(ws, L.w);
     float* logits = at<float>(ws, L.logits);
 
-    // weights for the tensor-core GEMMs
+    // the tensor-core GEMMs read the weights as given: bf16 (kind::f16) or,
+    // for fp32 problems, fp32 read as TF32 (kind::tf32)
     const void* ew = expert_w;
     const void* sw = shared_w;
-    if (f32) {
-        MOE_TRY(run_cast(expert_w, at<void>(ws, L.w_bf16), E * 3 * I * H, s));
-        ew = at<void>(ws, L.w_bf16);
-        if (S) {
-            MOE_TRY(run_cast(shared_w, at<void>(ws, L.ws_bf16), 3 * I * H, s));
-            sw = at<void>(ws, L.ws_bf16);
-        }
-    }
+    const ElemType et = f32 ? kF32 : kBF16;
 
     // 1. route
     MOE_TRY(run_route(p, x, gate_w, bias, logits, at<int32_t>(ws, L.rcount), idx, w, false,
@@ -1241,28 +1248,27 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
                          at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets), sg, nmax, sd,
                          nmax_dn, pos, src, row_w, status, s));
 
-    // 3. token rows for the gate/up GEMM: bf16 problems gather them inside the
-    //    GEMM (from x, by src); fp32 problems copy them into x_perm as bf16.
-    //    The scatter-add combine also needs its fp32 accumulator zeroed.
-    __nv_bfloat16* x_perm = at<__nv_bfloat16>(ws, L.x_perm);
+    // 3. token rows for the gate/up GEMM: gathered inside the GEMM (from x, by
+    //    src) or copied into x_perm in expert order by the gather kernel (the
+    //    problem dtype: fp32 rows for fp32 problems).  The scatter-add combine
+    //    also needs its fp32 accumulator zeroed.
+    void* x_perm = at<void>(ws, L.x_perm);
     // launches from here on may start while their predecessor finishes: each
     // waits for it before reading its outputs, and reads nothing earlier than
     // that except what was complete before the predecessor could start
     const bool pdl = pdl_enabled();
     const bool atomic_combine = combine_atomic();
     float* out_acc = atomic_combine ? at<float>(ws, L.out_acc) : nullptr;
-    __nv_bfloat16* y_perm = at<__nv_bfloat16>(ws, L.y_perm);
+    void* y_perm = at<void>(ws, L.y_perm);
     const bool gather_in_gemm = !f32 && fused_gather(nmax);
-    const void* x_b = x;
     if (f32) {
-        MOE_TRY((run_gather<float, __nv_bfloat16>(static_cast<const float*>(x), T, p->H, p->top_k,
-                                                  pos, T * k, x_perm, at<__nv_bfloat16>(ws, L.x_bf16),
-                                                  out_acc, s, pdl)));
-        x_b = at<void>(ws, L.x_bf16);
+        MOE_TRY((run_gather<float, float>(static_cast<const float*>(x), T, p->H, p->top_k, pos,
+                                          T * k, static_cast<float*>(x_perm), nullptr, out_acc, s,
+                                          pdl)));
     } else if (!gather_in_gemm) {
-        MOE_TRY((run_gather<__nv_bfloat16, __nv_bfloat16>(static_cast<const __nv_bfloat16*>(x), T,
-                                                          p->H, p->top_k, pos, T * k, x_perm,
-                                                          nullptr, out_acc, s, pdl)));
+        MOE_TRY((run_gather<__nv_bfloat16, __nv_bfloat16>(
+            static_cast<const __nv_bfloat16*>(x), T, p->H, p->top_k, pos, T * k,
+            static_cast<__nv_bfloat16*>(x_perm), nullptr, out_acc, s, pdl)));
     } else if (out_acc) {
         if (cudaMemsetAsync(out_acc, 0, static_cast<size_t>(T) * H * sizeof(float), s) !=
             cudaSuccess)
@@ -1270,16 +1276,16 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
     }
 
     // 4. grouped gate/up GEMM + clamp + SwiGLU (routed experts, then shared)
-    __nv_bfloat16* h = at<__nv_bfloat16>(ws, L.h_perm);
+    void* h = at<void>(ws, L.h_perm);
     const int64_t h_rows = T * (k + S);
     const int nseg = static_cast<int>(E + S);
     {
         GemmArgs a = base_args(status);
-        if (!make_tmap_gateup(&a.tmA0, ew, E * 3, I, H)) return MOE_ERR_CUDA;
-        if (!make_tmap_rows(a.tmB0, x_perm, T * k, H)) return MOE_ERR_CUDA;
+        if (!make_tmap_gateup(&a.tmA0, ew, E * 3, I, H, et)) return MOE_ERR_CUDA;
+        if (!make_tmap_rows(a.tmB0, x_perm, T * k, H, et)) return MOE_ERR_CUDA;
         if (S) {
-            if (!make_tmap_gateup(&a.tmA1, sw, 3, I, H)) return MOE_ERR_CUDA;
-            if (!make_tmap_rows(a.tmB1, x_b, T, H)) return MOE_ERR_CUDA;
+            if (!make_tmap_gateup(&a.tmA1, sw, 3, I, H, et)) return MOE_ERR_CUDA;
+            if (!make_tmap_rows(a.tmB1, x, T, H, et)) return MOE_ERR_CUDA;
         } else {
             a.tmA1 = a.tmA0;
             for (int j = 0; j < kNumBoxSizes; ++j) a.tmB1[j] = a.tmB0[j];
@@ -1303,8 +1309,12 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
         // launch is an ordinary one)
         const bool pdl_gu = pdl && !(gather_in_gemm && out_acc);
         expert_gemm_launch_args(a, true);
-        MOE_TRY(launch_gemm<EPI_SWIGLU>(nmax, 2, a, max_tiles(h_rows, nseg, nmax, I), s,
-                                        "expert_gate_up_gemm", pdl_gu));
+        if (f32)
+            MOE_TRY(launch_gemm_tf32<EPI_SWIGLU>(nmax, 2, a, max_tiles(h_rows, nseg, nmax, I), s,
+                                                 "expert_gate_up_gemm_tf32", pdl_gu));
+        else
+            MOE_TRY(launch_gemm<EPI_SWIGLU>(nmax, 2, a, max_tiles(h_rows, nseg, nmax, I), s,
+                                            "expert_gate_up_gemm", pdl_gu));
     }
     // 5. grouped down GEMM; its epilogue applies the routing weight and either
     //    stores the weighted rows (gather combine) or scatter-adds them into the
@@ -1312,10 +1322,10 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
     {
         GemmArgs a = base_args(status);
         const int mb = pick_down_mb(nmax_dn);
-        if (!make_tmap_down(&a.tmA0, ew, E * 3 * I, H, mb)) return MOE_ERR_CUDA;
-        if (!make_tmap_rows(a.tmB0, h, h_rows, I)) return MOE_ERR_CUDA;
+        if (!make_tmap_down(&a.tmA0, ew, E * 3 * I, H, mb, et)) return MOE_ERR_CUDA;
+        if (!make_tmap_rows(a.tmB0, h, h_rows, I, et)) return MOE_ERR_CUDA;
         if (S) {
-            if (!make_tmap_down(&a.tmA1, sw, 3 * I, H, mb)) return MOE_ERR_CUDA;
+            if (!make_tmap_down(&a.tmA1, sw, 3 * I, H, mb, et)) return MOE_ERR_CUDA;
         } else {
             a.tmA1 = a.tmA0;
         }
@@ -1336,12 +1346,21 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
         expert_gemm_launch_args(a, false);
         if (atomic_combine) {
             a.out = out_acc;
-            MOE_TRY(launch_gemm<EPI_DOWN_ATOMIC>(nmax_dn, mb, a, tiles, s,
-                                                 "expert_down_combine_gemm", pdl));
+            if (f32)
+                MOE_TRY(launch_gemm_tf32<EPI_DOWN_ATOMIC>(nmax_dn, mb, a, tiles, s,
+                                                          "expert_down_combine_gemm_tf32", pdl));
+            else
+                MOE_TRY(launch_gemm<EPI_DOWN_ATOMIC>(nmax_dn, mb, a, tiles, s,
+                                                     "expert_down_combine_gemm", pdl));
         } else {
             a.out = y_perm;
-            MOE_TRY(launch_gemm<EPI_DOWN_STORE>(nmax_dn, mb, a, tiles, s, "expert_down_gemm",
-                                                pdl));
+            a.out_f32 = f32 ? 1 : 0;  // fp32 problems: fp32 weighted rows
+            if (f32)
+                MOE_TRY(launch_gemm_tf32<EPI_DOWN_STORE>(nmax_dn, mb, a, tiles, s,
+                                                         "expert_down_gemm_tf32", pdl));
+            else
+                MOE_TRY(launch_gemm<EPI_DOWN_STORE>(nmax_dn, mb, a, tiles, s, "expert_down_gemm",
+                                                    pdl));
         }
     }
     // 6. token-order output
@@ -1352,10 +1371,10 @@ int32_t moe_forward(const moe_problem* p, const void* x, const void* gate_w, con
     }
     const int64_t shared_row0 = S ? T * k : -1;
     if (f32)
-        return run_gather_sum(y_perm, pos, T, p->H, p->top_k, T * k, shared_row0,
-                              static_cast<float*>(out), status, s, pdl);
-    return run_gather_sum(y_perm, pos, T, p->H, p->top_k, T * k, shared_row0,
-                          static_cast<__nv_bfloat16*>(out), status, s, pdl);
+        return run_gather_sum(static_cast<const float*>(y_perm), pos, T, p->H, p->top_k, T * k,
+                              shared_row0, static_cast<float*>(out), status, s, pdl);
+    return run_gather_sum(static_cast<const __nv_bfloat16*>(y_perm), pos, T, p->H, p->top_k,
+                          T * k, shared_row0, static_cast<__nv_bfloat16*>(out), status, s, pdl);
 }
 
 }  // extern "C"
@@ -1602,8 +1621,9 @@ int32_t moe_forward_fp8(const moe_problem* p, const void* x, const void* gate_w,
                                                 "expert_down_gemm_fp8", pdl));
     }
     // 6. fixed-order combine into token order
-    return run_gather_sum(y_perm, pos, T, p->H, p->top_k, T * k, S ? T * k : -1,
-                          static_cast<__nv_bfloat16*>(out), status, s, pdl);
+    return run_gather_sum(static_cast<const __nv_bfloat16*>(y_perm), pos, T, p->H, p->top_k,
+                          T * k, S ? T * k : -1, static_cast<__nv_bfloat16*>(out), status, s,
+                          pdl);
 }
 
 int32_t moe_read_device_status(const void* ws, int32_t* status_out, void* stream) {

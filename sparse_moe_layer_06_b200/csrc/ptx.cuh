@@ -347,6 +347,28 @@ __device__ __forceinline__ void mma_fp8(uint32_t d_tmem, uint64_t a_desc, uint64
     }
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::tf32 (fp32 inputs read as TF32,
+// fp32 accumulate).
+template <int CG = 1>
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+    if constexpr (CG == 2) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+            : "memory");
+    }
+}
+
 // Two floats to two E4M3 codes (round to nearest even, saturating to +-448):
 // the low byte holds `lo`, the high byte `hi`.
 __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
@@ -416,12 +438,40 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
     return d;
 }
 
+// The same for the 128-byte swizzle with 32-byte atoms (layout type 1): each
+// 128-byte row's four 32-byte chunks are permuted by (row mod 4), so the
+// swizzle repeats every 4 rows.  This is the only MN-major layout TF32
+// operands accept.
+__device__ __forceinline__ uint64_t smem_desc_sw128_32b(uint32_t saddr, uint32_t lbo_bytes,
+                                                        uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= 1ull << 46;
+    d |= 1ull << 61;
+    return d;
+}
+
 // Instruction descriptor for kind::f8f6f4 with E4M3 A/B and fp32 D (format
 // code 0 = E4M3 for both operands).
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(uint32_t M, uint32_t N, uint32_t a_mn_major,
                                                       uint32_t b_mn_major) {
     return (1u << 4) | (a_mn_major << 15) | (b_mn_major << 16) | ((N >> 3) << 17) |
            ((M >> 4) << 24);
+}
+
+// Instruction descriptor for kind::tf32 with TF32 A/B (format code 2) and
+// fp32 D.
+__host__ __device__ constexpr uint32_t idesc_tf32_f32(uint32_t M, uint32_t N, uint32_t a_mn_major,
+                                                      uint32_t b_mn_major) {
+    return (1u << 4)                 // D format: f32
+           | (2u << 7)               // A format: tf32
+           | (2u << 10)              // B format: tf32
+           | (a_mn_major << 15)      // A major-ness
+           | (b_mn_major << 16)      // B major-ness
+           | ((N >> 3) << 17)        // N / 8
+           | ((M >> 4) << 24);       // M / 16
 }
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.

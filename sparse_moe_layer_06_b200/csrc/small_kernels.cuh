@@ -428,17 +428,36 @@ __global__ void combine_kernel(const T* __restrict__ y_perm, const int32_t* __re
 // Fixed-order combine of weighted expert rows (the down GEMM already applied
 // the routing weights): out[t] = sum_j y[pos[t,j]] (j = 0..k-1 in slot order)
 // + y[shared_row0 + t] when shared_row0 >= 0, summed in fp32.  One warp per
-// (token, 512-value segment of H): 16-byte vectors, two per lane in flight per
-// row, so even a few tokens spread over many warps.
+// (token, segment of 64 16-byte vectors of H): two vectors per lane in flight
+// per row, so even a few tokens spread over many warps.  y is bf16 (8 values
+// per vector) or fp32 (4 values per vector).
 constexpr int kSegVecs = 64;  // 16-byte vectors per warp segment
 
-template <typename TOut, int kBatch>
-__global__ void gather_sum_kernel(const __nv_bfloat16* __restrict__ y,
-                                  const int32_t* __restrict__ pos, int64_t T, int H, int k,
-                                  int64_t n_rows, int64_t shared_row0, TOut* __restrict__ out,
-                                  int32_t* status) {
+template <typename TIn>
+__device__ __forceinline__ void add_vec(float (&acc)[16 / sizeof(TIn)], const uint4& q) {
+    if constexpr (sizeof(TIn) == 2) {
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(h2[e]);
+            acc[2 * e] += f.x;
+            acc[2 * e + 1] += f.y;
+        }
+    } else {
+        acc[0] += __uint_as_float(q.x);
+        acc[1] += __uint_as_float(q.y);
+        acc[2] += __uint_as_float(q.z);
+        acc[3] += __uint_as_float(q.w);
+    }
+}
+
+template <typename TIn, typename TOut, int kBatch>
+__global__ void gather_sum_kernel(const TIn* __restrict__ y, const int32_t* __restrict__ pos,
+                                  int64_t T, int H, int k, int64_t n_rows, int64_t shared_row0,
+                                  TOut* __restrict__ out, int32_t* status) {
+    constexpr int kVE = 16 / static_cast<int>(sizeof(TIn));  // values per 16-byte vector
     const int lane = threadIdx.x & 31;
-    const int nvec = H / 8;
+    const int nvec = H / kVE;
     const int nseg = (nvec + kSegVecs - 1) / kSegVecs;
     ptx::grid_dep_wait();  // the rows come from the previous launch
     const int64_t gw = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -457,18 +476,9 @@ __global__ void gather_sum_kernel(const __nv_bfloat16* __restrict__ y,
         const int v0 = seg * kSegVecs;
         const int va = v0 + lane, vb = v0 + 32 + lane;
         const bool oka = va < nvec, okb = vb < nvec;
-        float acc_a[8], acc_b[8];
+        float acc_a[kVE], acc_b[kVE];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc_a[e] = acc_b[e] = 0.0f;
-        auto add8 = [](float (&acc)[8], const uint4& q) {
-            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&q);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(h2[e]);
-                acc[2 * e] += f.x;
-                acc[2 * e + 1] += f.y;
-            }
-        };
+        for (int e = 0; e < kVE; ++e) acc_a[e] = acc_b[e] = 0.0f;
         // rows in slot order (the shared expert's last), loaded kBatch at a
         // time before any is added; the additions stay in slot order
         const int n_rows_t = k + (shared_row0 >= 0 ? 1 : 0);
@@ -487,21 +497,29 @@ __global__ void gather_sum_kernel(const __nv_bfloat16* __restrict__ y,
             }
 #pragma unroll
             for (int b = 0; b < kBatch; ++b) {
-                if (has[b] && oka) add8(acc_a, qa[b]);
-                if (has[b] && okb) add8(acc_b, qb[b]);
+                if (has[b] && oka) add_vec<TIn>(acc_a, qa[b]);
+                if (has[b] && okb) add_vec<TIn>(acc_b, qb[b]);
             }
         }
-        auto put = [&](const float (&acc)[8], int v) {
-            if constexpr (sizeof(TOut) == 2) {
+        auto put = [&](const float (&acc)[kVE], int v) {
+            TOut* o = out + t * H + static_cast<int64_t>(v) * kVE;
+            if constexpr (sizeof(TOut) == 2 && kVE == 8) {
                 uint4 q;
                 __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&q);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) h2[e] = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
-                reinterpret_cast<uint4*>(out + t * H)[v] = q;
+                *reinterpret_cast<uint4*>(o) = q;
+            } else if constexpr (sizeof(TOut) == 2) {
+                uint2 q;
+                __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&q);
+                h2[0] = __floats2bfloat162_rn(acc[0], acc[1]);
+                h2[1] = __floats2bfloat162_rn(acc[2], acc[3]);
+                *reinterpret_cast<uint2*>(o) = q;
             } else {
-                float4* o = reinterpret_cast<float4*>(out + t * H);
-                o[2 * v] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-                o[2 * v + 1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+#pragma unroll
+                for (int e = 0; e < kVE; e += 4)
+                    *reinterpret_cast<float4*>(o + e) =
+                        make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
             }
         };
         if (oka) put(acc_a, va);
@@ -610,12 +628,5 @@ __global__ void quantize_cols_e4m3_kernel(const T* __restrict__ in, int64_t mat_
     scale[id] = sc;
 }
 
-__global__ void cast_f32_bf16_kernel(const float* __restrict__ in, __nv_bfloat16* __restrict__ out,
-                                     int64_t n) {
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        out[i] = __float2bfloat16_rn(in[i]);
-    }
-}
 
 }  // namespace moe

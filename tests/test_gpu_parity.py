@@ -5,7 +5,7 @@ import pytest
 import torch
 
 import oracle
-from parity_util import (OUT_TOL, assert_close_out, check_routing, forward_parity,
+from parity_util import (OUT_TOL, assert_close_out, check_routing, forward_parity, out_tol,
                          to_cpu_inputs)
 from sparse_moe_layer_06_b200 import moe
 from sparse_moe_layer_06_b200.workloads import MoEConfig, make_inputs
@@ -170,7 +170,7 @@ def test_grouped_ffn_matches_oracle(shape, dtype):
     torch.cuda.synchronize()
     assert moe.moe_read_device_status(ws) == 0
     ref = oracle.expert_rows(ci["x"], ci["expert_w"], None, src, row_expert, c.clip_limit)
-    assert_close_out(y.float().cpu().numpy(), ref, "grouped ffn")
+    assert_close_out(y.float().cpu().numpy(), ref, "grouped ffn", out_tol(c))
 
 
 def test_grouped_ffn_clamp_saturated():
@@ -259,7 +259,9 @@ def test_forward_fp32_tiny_config():
     inp = make_inputs(c, seed=0, device=DEV)
     out, idx, w = run_forward(c, inp)
     assert out.dtype == torch.float32
-    forward_parity(inp, c, out, idx, w)
+    # TF32 expert GEMMs: checked to the fp32 bound (a quarter of the bf16 one)
+    _, err, scale = forward_parity(inp, c, out, idx, w)
+    print(f"tiny fp32 layer: max err {err:.3e} of max |out| {scale:.3e} ({err / scale:.2e})")
 
 
 def test_forward_all_tokens_to_two_experts():
