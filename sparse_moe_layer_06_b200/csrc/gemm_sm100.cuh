@@ -303,6 +303,67 @@ __device__ __forceinline__ float clamp_keep_nan(float v, float lim) {
     return v > lim ? lim : (v < -lim ? -lim : v);
 }
 
+// Output rows from the accumulator layout (one output column m per lane, 16
+// token rows per chunk): the lanes of a pair (m even, m + 1) store 2-element
+// units, the even lane those of the even token rows, the odd lane those of the
+// odd ones.  One shuffle carries two bf16 (or four E4M3) values, so a chunk
+// of 16 token rows takes 4 (2) shuffles and 8 stores per lane.  Each value is
+// rounded on its own, as a single conversion would round it.
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+    const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&p);
+}
+
+// bf16 rows: a[j] is this lane's value for token row j of the chunk; row j
+// starts at element `row0 + j * ld` (row0 = the chunk's first row at the even
+// lane's column).  ok(j): whether token row j is stored.
+template <typename OkFn>
+__device__ __forceinline__ void store_pairs_bf16(__nv_bfloat16* out, size_t row0, size_t ld,
+                                                 const float (&a)[16], bool odd, OkFn ok) {
+#pragma unroll
+    for (int j = 0; j < 16; j += 4) {
+        const uint32_t own = bf16x2_bits(odd ? a[j + 1] : a[j], odd ? a[j + 3] : a[j + 2]);
+        const uint32_t snd = bf16x2_bits(odd ? a[j] : a[j + 1], odd ? a[j + 2] : a[j + 3]);
+        const uint32_t rcv = __shfl_xor_sync(0xffffffffu, snd, 1);
+        const uint32_t ev = odd ? rcv : own;  // the even lane's values of the two rows
+        const uint32_t od = odd ? own : rcv;  // the odd lane's
+        const int r = j + (odd ? 1 : 0);
+        if (ok(r))
+            *reinterpret_cast<uint32_t*>(out + row0 + r * ld) = __byte_perm(ev, od, 0x5410);
+        if (ok(r + 2))
+            *reinterpret_cast<uint32_t*>(out + row0 + (r + 2) * ld) = __byte_perm(ev, od, 0x7632);
+    }
+}
+
+// E4M3 rows, as store_pairs_bf16 (byte offsets).
+template <typename OkFn>
+__device__ __forceinline__ void store_pairs_e4m3(uint8_t* out, size_t row0, size_t ld,
+                                                 const float (&a)[16], bool odd, OkFn ok) {
+#pragma unroll
+    for (int j = 0; j < 16; j += 8) {
+        uint32_t own = 0, snd = 0;
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+            const int b = j + 4 * g;
+            own |= static_cast<uint32_t>(ptx::e4m3x2(odd ? a[b + 1] : a[b], odd ? a[b + 3] : a[b + 2]))
+                   << (16 * g);
+            snd |= static_cast<uint32_t>(ptx::e4m3x2(odd ? a[b] : a[b + 1], odd ? a[b + 2] : a[b + 3]))
+                   << (16 * g);
+        }
+        const uint32_t rcv = __shfl_xor_sync(0xffffffffu, snd, 1);
+        const uint32_t ev = odd ? rcv : own;
+        const uint32_t od = odd ? own : rcv;
+        const int r = j + (odd ? 1 : 0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            // byte q of each lane's word: token row r + 2q
+            if (ok(r + 2 * q))
+                *reinterpret_cast<uint16_t*>(out + row0 + (r + 2 * q) * ld) =
+                    static_cast<uint16_t>(__byte_perm(ev, od, q | ((4 + q) << 4)));
+        }
+    }
+}
+
 template <int EPI, int NMAX, int MB, int ET, bool PAIR, int GW>
 __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, ET, PAIR, GW>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmArgs args) {
@@ -760,6 +821,19 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, ET, PAIR, GW>::kThreads
         ptx::grid_dep_wait();  // row metadata and outputs are shared with earlier launches
         uint32_t acc = 0, acc_phase = 0;
         uint32_t mi = 0, meta_phase = 0;
+        // hands accumulator buffer `acc` back to the MMA warp once this warp's
+        // TMEM reads of it have completed (PAIR: on the leader CTA, which
+        // waits for both CTAs)
+        auto release_acc = [&]() {
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if constexpr (PAIR)
+                    ptx::mbar_arrive_cluster(ptx::mapa_shared(ptx::smem_u32(&acce_bar[acc]), 0));
+                else
+                    ptx::mbar_arrive(&acce_bar[acc]);
+            }
+        };
         for (int t = unit; t < total_tiles; t += units) {
             TileInfo ti;
             const int ks = t % ksplit;
@@ -797,6 +871,29 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, ET, PAIR, GW>::kThreads
                 mi ^= 1;
                 if (mi == 0) meta_phase ^= 1;
             }
+            // FP8 channel scales of this lane's rows, fetched before the
+            // accumulator is ready (under the main loop): gate/up: the gate
+            // and up scales of row m; down: h scale x weight-column scale of
+            // each sub-tile's row
+            static_assert(MB <= 2, "at most two 128-row sub-tiles");
+            float ch0 = 1.0f, ch1 = 1.0f;
+            if constexpr (FP8 && C::kSwiGLU) {
+                const int m = ti.blk * 128 + row_in_tile;
+                const float* sc = ti.special ? args.scale_w_special
+                                             : args.scale_w + static_cast<size_t>(ti.seg) * 2 *
+                                                                  args.M_total;
+                if (m < args.M_total) {
+                    ch0 = __ldg(sc + m);
+                    ch1 = __ldg(sc + args.M_total + m);
+                }
+            } else if constexpr (FP8 && C::kDown) {
+                const float* sc = ti.special ? args.scale_w_special
+                                             : args.scale_w + static_cast<size_t>(ti.seg) *
+                                                                  args.M_total;
+                const int m0 = ti.blk * MB * 128 + row_in_tile;
+                if (m0 < args.M_total) ch0 = args.h_scale * __ldg(sc + m0);
+                if (MB > 1 && m0 + 128 < args.M_total) ch1 = args.h_scale * __ldg(sc + m0 + 128);
+            }
             if (!ptx::mbar_wait(&accf_bar[acc], acc_phase, abort_flag)) {
                 fail(DEV_ERR_TIMEOUT);
                 break;
@@ -807,31 +904,30 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, ET, PAIR, GW>::kThreads
             if constexpr (C::kSwiGLU) {
                 // h = silu(clamp(g)) * clamp(u) on this warp's 16-column chunks;
                 // the next chunk's TMEM loads are in flight while one is
-                // computed.  Lanes pair up (i, i+1) so each store is a bf16x2.
+                // computed.
                 const int m = ti.blk * 128 + row_in_tile;
-                const bool m_ok = m < args.M_total;  // I is even: lane pairs agree
-                const bool odd = lane & 1;
-                const int m_pair = m - (odd ? 1 : 0);
+                const bool m_ok = m < args.M_total;
                 __nv_bfloat16* hout = reinterpret_cast<__nv_bfloat16*>(args.out);
-                // FP8: gate and up channel scales of this lane's row
-                float sg = 1.0f, su = 1.0f;
-                if constexpr (FP8) {
-                    const float* sc = ti.special ? args.scale_w_special
-                                                 : args.scale_w + static_cast<size_t>(ti.seg) * 2 *
-                                                                      args.M_total;
-                    if (m_ok) {
-                        sg = __ldg(sc + m);
-                        su = __ldg(sc + args.M_total + m);
-                    }
-                }
+                const float sg = ch0, su = ch1;  // FP8: gate and up channel scales
                 auto emit = [&](float (&g)[16], float (&u)[16], int c0) {
                     float hv[16];
+                    float ts16[16];  // FP8 token scales, read before the stores
+                    if constexpr (FP8) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float4 t4 = reinterpret_cast<const float4*>(w_wt + c0)[q];
+                            ts16[4 * q] = t4.x;
+                            ts16[4 * q + 1] = t4.y;
+                            ts16[4 * q + 2] = t4.z;
+                            ts16[4 * q + 3] = t4.w;
+                        }
+                    }
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         float gin = g[j], uin = u[j];
                         if constexpr (FP8) {
                             // token scale (per column) x channel scale (per lane)
-                            const float ts = w_wt[c0 + j];
+                            const float ts = ts16[j];
                             gin *= ts * sg;
                             uin *= ts * su;
                         }
@@ -854,28 +950,15 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, ET, PAIR, GW>::kThreads
                         }
                         return;
                     }
-#pragma unroll
-                    for (int j = 0; j < 16; j += 2) {
-                        // even lane: (my h, partner's h) of column j;
-                        // odd lane: (partner's h, my h) of column j+1
-                        const float mine = odd ? hv[j + 1] : hv[j];
-                        const float send = odd ? hv[j] : hv[j + 1];
-                        const float other = __shfl_xor_sync(0xffffffffu, send, 1);
-                        const int col = c0 + j + (odd ? 1 : 0);
-                        const float lo = odd ? other : mine;
-                        const float hi = odd ? mine : other;
-                        if (m_ok && col < ti.n_valid) {
-                            const size_t o =
-                                static_cast<size_t>(ti.out_row + col) * args.out_ld + m_pair;
-                            if constexpr (FP8) {
-                                *reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(args.out) +
-                                                             o) = ptx::e4m3x2(lo, hi);
-                            } else {
-                                *reinterpret_cast<__nv_bfloat162*>(hout + o) =
-                                    __floats2bfloat162_rn(lo, hi);
-                            }
-                        }
-                    }
+                    // lane pairs (I is a multiple of 64: a pair agrees on m_ok)
+                    const bool odd = lane & 1;
+                    const size_t ld = static_cast<size_t>(args.out_ld);
+                    const size_t row0 = static_cast<size_t>(ti.out_row + c0) * ld + (m & ~1);
+                    auto ok = [&](int r) { return m_ok && c0 + r < ti.n_valid; };
+                    if constexpr (FP8)
+                        store_pairs_e4m3(reinterpret_cast<uint8_t*>(args.out), row0, ld, hv, odd, ok);
+                    else
+                        store_pairs_bf16(hout, row0, ld, hv, odd, ok);
                 };
                 float g0[16], u0[16], g1[16], u1[16];
                 int c0 = half * 16;  // this warp's chunks: c0, c0 + 32, ...
@@ -909,92 +992,113 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, ET, PAIR, GW>::kThreads
                     ptx::reg_fence(u0);
                 }
             } else {
+                // Per sub-tile, this warp's 16-column chunks are read from TMEM
+                // in batches of up to five (80 registers) behind one wait.  The
+                // down GEMMs hand the accumulator back to the MMA warp as soon
+                // as their last batch is in registers, so the next tile's MMAs
+                // run under the scaling and stores of that batch.
+                constexpr int kCW = (NMAX + 31) / 32;       // chunks per warp and sub-tile
+                constexpr int kNB = (kCW + 4) / 5;          // batches per sub-tile
+                constexpr int kBC = (kCW + kNB - 1) / kNB;  // chunks per batch
+                auto emit_chunk = [&](const float (&v)[16], int c0, int m, bool m_ok,
+                                      float lane_scale) {
+                    // The chunk's column weights (and tokens) are read into
+                    // registers before its first store: the output pointer is
+                    // generic, so a read of the metadata placed after a store
+                    // could not be moved above it and every column would wait
+                    // out a full memory round trip.
+                    float cw[16];
+                    if constexpr (C::kMeta) {
+                        // (16-byte loads: the metadata buffers and c0 are
+                        // 64-byte aligned)
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float4 w4 = reinterpret_cast<const float4*>(w_wt + c0)[q];
+                            cw[4 * q] = w4.x;
+                            cw[4 * q + 1] = w4.y;
+                            cw[4 * q + 2] = w4.z;
+                            cw[4 * q + 3] = w4.w;
+                        }
+                    }
+                    if constexpr (EPI == EPI_DOWN_ATOMIC) {
+                        float* oacc = reinterpret_cast<float*>(args.out);
+                        // each accumulator element takes top_k + 1 additions spread
+                        // over the whole launch: keep its lines in L2 between them
+                        const uint64_t pol_acc = args.l2_hints ? ptx::policy_evict_last()
+                                                               : ptx::policy_evict_normal();
+                        int ct[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) ct[j] = w_tok[c0 + j];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int c = c0 + j;
+                            if (m_ok && c < ti.n_valid) {
+                                const int tok = ct[j];
+                                if (static_cast<unsigned>(tok) <
+                                    static_cast<unsigned>(args.n_tokens)) {
+                                    ptx::red_add_f32(
+                                        oacc + static_cast<size_t>(tok) * args.out_ld + m,
+                                        cw[j] * v[j], pol_acc);
+                                } else {
+                                    set_device_error(args.status, DEV_ERR_BAD_INDEX);
+                                }
+                            }
+                        }
+                    } else if (EPI == EPI_DOWN_STORE && !args.out_f32) {
+                        // weighted bf16 rows, stored by lane pairs (H is a
+                        // multiple of 64: a pair agrees on m_ok)
+                        float a[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) a[j] = v[j] * lane_scale * cw[j];
+                        const size_t ld = static_cast<size_t>(args.out_ld);
+                        const size_t row0 =
+                            static_cast<size_t>(ti.out_row + c0) * ld + (m & ~1);
+                        store_pairs_bf16(reinterpret_cast<__nv_bfloat16*>(args.out), row0, ld, a,
+                                         (lane & 1) != 0,
+                                         [&](int r) { return m_ok && c0 + r < ti.n_valid; });
+                    } else if (m_ok) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            if (c0 + j < ti.n_valid) {
+                                const size_t o =
+                                    static_cast<size_t>(ti.out_row + c0 + j) * args.out_ld + m;
+                                if constexpr (EPI == EPI_LOGITS) {
+                                    reinterpret_cast<float*>(args.out)[o + ks * args.split_stride] =
+                                        v[j];
+                                } else {
+                                    reinterpret_cast<float*>(args.out)[o] = v[j] * cw[j];
+                                }
+                            }
+                        }
+                    }
+                };
 #pragma unroll 1
                 for (int sub = 0; sub < MB; ++sub) {
                     const int m = (ti.blk * MB + sub) * 128 + row_in_tile;
                     const bool m_ok = m < args.M_total;
                     // FP8: h scale x this lane's weight-column scale
-                    float lane_scale = 1.0f;
-                    if constexpr (FP8 && C::kDown) {
-                        const float* sc = ti.special ? args.scale_w_special
-                                                     : args.scale_w + static_cast<size_t>(ti.seg) *
-                                                                          args.M_total;
-                        if (m_ok) lane_scale = args.h_scale * __ldg(sc + m);
-                    }
-                    for (int c0 = half * 16; c0 < ti.n_mma; c0 += 32) {
-                        float v[16];
-                        ptx::tmem_ld16(tbase + sub * NMAX + c0, v);
+                    const float lane_scale = sub == 0 ? ch0 : ch1;
+#pragma unroll 1
+                    for (int b = 0; b < kNB; ++b) {
+                        float v[kBC][16];
+#pragma unroll
+                        for (int i = 0; i < kBC; ++i) {
+                            const int c0 = half * 16 + 32 * (b * kBC + i);
+                            if (c0 < ti.n_mma) ptx::tmem_ld16(tbase + sub * NMAX + c0, v[i]);
+                        }
                         ptx::tmem_ld_wait();
-                        ptx::reg_fence(v);
-                        if constexpr (EPI == EPI_DOWN_ATOMIC) {
-                            float* oacc = reinterpret_cast<float*>(args.out);
-                            // each accumulator element takes top_k + 1 additions spread
-                            // over the whole launch: keep its lines in L2 between them
-                            const uint64_t pol_acc = args.l2_hints ? ptx::policy_evict_last()
-                                                                   : ptx::policy_evict_normal();
 #pragma unroll
-                            for (int j = 0; j < 16; ++j) {
-                                const int c = c0 + j;
-                                if (m_ok && c < ti.n_valid) {
-                                    const int tok = w_tok[c];
-                                    if (static_cast<unsigned>(tok) <
-                                        static_cast<unsigned>(args.n_tokens)) {
-                                        ptx::red_add_f32(
-                                            oacc + static_cast<size_t>(tok) * args.out_ld + m,
-                                            w_wt[c] * v[j], pol_acc);
-                                    } else {
-                                        set_device_error(args.status, DEV_ERR_BAD_INDEX);
-                                    }
-                                }
-                            }
-                        } else if (EPI == EPI_DOWN_STORE && !args.out_f32) {
-                            // weighted bf16 rows; lanes pair up (h, h+1) so each
-                            // store is a bf16x2 (H is even: lane pairs agree on m_ok)
-                            const bool odd = lane & 1;
-                            const int m_pair = m - (odd ? 1 : 0);
-                            __nv_bfloat16* yout = reinterpret_cast<__nv_bfloat16*>(args.out);
+                        for (int i = 0; i < kBC; ++i) ptx::reg_fence(v[i]);
+                        if (C::kDown && sub == MB - 1 && b == kNB - 1) release_acc();
 #pragma unroll
-                            for (int j = 0; j < 16; j += 2) {
-                                const int c = c0 + j;
-                                const float a0 = v[j] * lane_scale * w_wt[c];
-                                const float a1 = v[j + 1] * lane_scale * w_wt[c + 1];
-                                const float mine = odd ? a1 : a0;
-                                const float send = odd ? a0 : a1;
-                                const float other = __shfl_xor_sync(0xffffffffu, send, 1);
-                                const int col = c + (odd ? 1 : 0);
-                                const __nv_bfloat162 pr = odd ? __floats2bfloat162_rn(other, mine)
-                                                              : __floats2bfloat162_rn(mine, other);
-                                if (m_ok && col < ti.n_valid) {
-                                    *reinterpret_cast<__nv_bfloat162*>(
-                                        yout + static_cast<size_t>(ti.out_row + col) * args.out_ld +
-                                        m_pair) = pr;
-                                }
-                            }
-                        } else if (m_ok) {
-#pragma unroll
-                            for (int j = 0; j < 16; ++j) {
-                                if (c0 + j < ti.n_valid) {
-                                    const size_t o =
-                                        static_cast<size_t>(ti.out_row + c0 + j) * args.out_ld + m;
-                                    if constexpr (EPI == EPI_LOGITS) {
-                                        reinterpret_cast<float*>(args.out)[o + ks * args.split_stride] =
-                                            v[j];
-                                    } else {
-                                        reinterpret_cast<float*>(args.out)[o] = v[j] * w_wt[c0 + j];
-                                    }
-                                }
-                            }
+                        for (int i = 0; i < kBC; ++i) {
+                            const int c0 = half * 16 + 32 * (b * kBC + i);
+                            if (c0 < ti.n_mma) emit_chunk(v[i], c0, m, m_ok, lane_scale);
                         }
                     }
                 }
             }
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                // PAIR: the accumulator buffer is free once both CTAs drained it
-                if constexpr (PAIR) ptx::mbar_arrive_cluster(ptx::mapa_shared(ptx::smem_u32(&acce_bar[acc]), 0));
-                else ptx::mbar_arrive(&acce_bar[acc]);
-            }
+            if constexpr (!C::kDown) release_acc();
             if (++acc == C::kAccStages) {
                 acc = 0;
                 acc_phase ^= 1;
