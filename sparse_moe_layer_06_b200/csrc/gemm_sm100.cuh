@@ -140,7 +140,8 @@ struct GemmArgs {
     float route_scale;
     int32_t route_keep_sum;
     // EPI_SWIGLU row gather: when gather_tok != nullptr, ordinary segments
-    // take their token rows straight from gather_src ([n_tokens, K] bf16) at
+    // take their token rows straight from gather_src ([n_tokens, K] bf16, or
+    // E4M3 codes in the gather-warp kernels) at
     // rows gather_tok[b_row + i] instead of from tmB0 (the permuted copy)
     const int32_t* gather_tok;
     const void* gather_src;
@@ -236,7 +237,7 @@ struct GemmCfg {
     static_assert((2 * kStages + 7) * 8 + 3 * 4 <= kBarrierBytes, "barrier area");
     // GW > 0 (EPI_SWIGLU with the row gather): that many more warps copy the
     // gathered token rows; the producer warp then only issues the weight copies
-    static_assert(GW == 0 || (EPI == EPI_SWIGLU && ET == 0 && !PAIR), "gather warps");
+    static_assert(GW == 0 || (EPI == EPI_SWIGLU && ET != 2 && !PAIR), "gather warps");
     static constexpr int kThreads = 32 * (2 + kEpiWarps + GW);
 };
 
@@ -530,8 +531,10 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, ET, PAIR, GW>::kThreads
             const CUtensorMap* tB = ti.special ? args.tmB1 : args.tmB0;
             const int a_base = ti.special ? 0 : ti.seg * args.a_seg_stride;
             const uint64_t pw = weight_policy(ti);
-            const bool gather =
-                C::kSwiGLU && ET == 0 && !PAIR && args.gather_tok != nullptr && !ti.special;
+            // (gathered rows: by the gather warps when GW > 0, bf16 or E4M3;
+            // by this warp itself, bf16 only)
+            const bool gather = C::kSwiGLU && (ET == 0 || GW > 0) && !PAIR &&
+                                args.gather_tok != nullptr && !ti.special;
             // GW > 0: the gather warps copy the rows; this warp only the weights
             const bool own_gather = gather && GW == 0;
             // token rows this CTA loads (PAIR: its half of the tile's columns)
@@ -749,7 +752,9 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, ET, PAIR, GW>::kThreads
         // group) and arrives once per stage on the full barrier, when its
         // copies have landed (at once for tiles it has no rows of)
         const int gw = warp - 2 - C::kEpiWarps;
-        const bf16_raw_ptr gsrc = reinterpret_cast<bf16_raw_ptr>(args.gather_src);
+        // (byte addressing: a stage holds 128 bytes of every row, 64 bf16 or
+        // 128 E4M3 values)
+        const uint8_t* gsrc = static_cast<const uint8_t*>(args.gather_src);
         ptx::grid_dep_wait();  // the row indices come from an earlier launch
         uint32_t stage = 0, phase = 0;
         bool ok = true;
@@ -771,7 +776,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, ET, PAIR, GW>::kThreads
                             r < ti.n_valid ? __ldg(args.gather_tok + ti.b_row + r) : -1;
                         s_goff[r] = static_cast<unsigned>(tok) <
                                             static_cast<unsigned>(args.n_tokens)
-                                        ? static_cast<int64_t>(tok) * args.K
+                                        ? static_cast<int64_t>(tok) * args.K * C::kElemBytes
                                         : int64_t(-1);
                     }
                 }
@@ -789,7 +794,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI, NMAX, MB, ET, PAIR, GW>::kThreads
                 if (gather) {
                     uint8_t* sB = ring + stage * C::kStageBytes + C::kABytes;
                     const int chunk = lane & 7;
-                    const bf16_raw_ptr base = gsrc + kb * C::kKStep + chunk * 8;
+                    const uint8_t* base = gsrc + kb * 128 + chunk * 16;
                     for (int g = gw; g < ngroups; g += GW) {
                         const int r0 = g * 16;
                         int64_t off[4];

@@ -566,6 +566,18 @@ int32_t launch_gemm_fp8(int nmax, int mb, const GemmArgs& a, int64_t max_tiles, 
     int grid = static_cast<int>(std::min<int64_t>(sm_count(), std::max<int64_t>(1, max_tiles)));
     const bool pair = use_pair() && nmax >= 64;
     if constexpr (EPI == EPI_SWIGLU) {
+        if (a.gather_tok != nullptr) {
+            // E4M3 token rows gathered by four gather warps
+            switch (nmax) {
+                case 16: return launch_gemm_n<EPI, 16, 2, 1, false, 4>(a, grid, s, name, false, pdl);
+                case 32: return launch_gemm_n<EPI, 32, 2, 1, false, 4>(a, grid, s, name, false, pdl);
+                case 64: return launch_gemm_n<EPI, 64, 2, 1, false, 4>(a, grid, s, name, false, pdl);
+                case 128: return launch_gemm_n<EPI, 128, 2, 1, false, 4>(a, grid, s, name, false, pdl);
+                case 160: return launch_gemm_n<EPI, 160, 2, 1, false, 4>(a, grid, s, name, false, pdl);
+                case 256: return launch_gemm_n<EPI, 256, 2, 1, false, 4>(a, grid, s, name, false, pdl);
+                default: return MOE_ERR_UNSUPPORTED;
+            }
+        }
         return launch_gemm_mb<EPI, 2, 1>(nmax, a, grid, s, name, pair, pdl);
     } else {
         static_assert(EPI == EPI_DOWN_STORE, "FP8 down GEMM uses the store epilogue");
@@ -648,8 +660,9 @@ bool combine_atomic() {
 }
 
 // Whether the gate/up GEMM gathers the routed token rows straight from x
-// (four gather warps, 16-byte cp.async into the swizzled stage; bf16
-// problems) instead of reading a permuted copy x_perm written by a separate
+// (four gather warps, 16-byte cp.async into the swizzled stage; bf16 rows,
+// or the E4M3 code rows of moe_forward_fp8) instead of reading a permuted copy
+// x_perm written by a separate
 // gather kernel.  Default: fused for token tiles of up to 160 rows (measured
 // 0.2-2% faster per layer at the Hy4 prefill and decode and the Hy3 batches,
 // from dropping the gather launch and the copy's DRAM round trip), the
@@ -1542,8 +1555,12 @@ int32_t moe_forward_fp8(const moe_problem* p, const void* x, const void* gate_w,
                    static_cast<const __nv_bfloat16*>(x), T, static_cast<int>(H), T, T, x_q, s_x));
     uint8_t* x_perm = at<uint8_t>(ws, L.x_perm);
     const bool pdl = pdl_enabled();
-    MOE_TRY((run_gather<uint8_t, uint8_t>(x_q, T, p->H, p->top_k, pos, T * k, x_perm, nullptr,
-                                          nullptr, s, pdl)));
+    // the gate/up GEMM's gather warps fetch the code rows straight from x_q
+    // (as for bf16 rows: tiles of up to 160 rows, MOE_FUSED_GATHER overrides)
+    const bool gather_in_gemm = fused_gather(nmax);
+    if (!gather_in_gemm)
+        MOE_TRY((run_gather<uint8_t, uint8_t>(x_q, T, p->H, p->top_k, pos, T * k, x_perm, nullptr,
+                                              nullptr, s, pdl)));
     // 4. gate/up on E4M3 codes; the epilogue applies token x channel scales,
     //    clamps, and writes h as E4M3 with the fixed power-of-two scale
     const double L_clip = p->clip_limit;
@@ -1581,6 +1598,11 @@ int32_t moe_forward_fp8(const moe_problem* p, const void* x, const void* gate_w,
         a.scale_w_special = shared_s_gu;
         a.h_scale = h_scale;
         a.h_scale_inv = 1.0f / h_scale;
+        if (gather_in_gemm) {
+            a.gather_tok = src;
+            a.gather_src = x_q;
+            a.n_tokens = static_cast<int32_t>(T);
+        }
         expert_gemm_launch_args(a, true);
         MOE_TRY(launch_gemm_fp8<EPI_SWIGLU>(nmax, 2, a, max_tiles(h_rows, nseg, nmax, I), s,
                                             "expert_gate_up_gemm_fp8", pdl));

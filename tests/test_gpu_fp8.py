@@ -151,6 +151,29 @@ def test_forward_fp8_saturating_clamp():
     oracle_fp8_parity(c, cpu, out, idx, w, list(range(c.T)))
 
 
+@pytest.mark.parametrize("shape", [dict(T=200, E=16, top_k=4, I=256),
+                                   dict(T=700, E=8, top_k=2, I=384)])
+def test_forward_fp8_row_gather_and_permuted_copy_agree(monkeypatch, shape):
+    """The gate/up GEMM takes the E4M3 token rows either straight from the
+    per-token codes by the gather warps (MOE_FUSED_GATHER=1; the default for
+    tiles of up to 160 rows) or from the permuted copy (MOE_FUSED_GATHER=0).
+    The two fill the same shared-memory tiles, so the layers are bit-identical;
+    both match the oracle.  The second shape has 175 rows per expert: tiles of
+    160 rows and ragged second chunks."""
+    c = MoEConfig("fp8_gather", H=512, num_shared=1, dtype=torch.bfloat16, x_std=1.0,
+                  w_std=0.05, routed_scale=2.827, clip_limit=10.0, **shape)
+    inp = make_inputs(c, seed=12, device=DEV)
+    cpu = to_cpu_inputs(inp)
+    outs = {}
+    for fg in ("1", "0"):
+        monkeypatch.setenv("MOE_FUSED_GATHER", fg)
+        out, idx, w, _, _ = run_fp8(c, inp)
+        oracle_fp8_parity(c, cpu, out, idx, w, list(range(0, c.T, 3)))
+        outs[fg] = (out, idx)
+    assert torch.equal(outs["1"][1], outs["0"][1])
+    assert torch.equal(outs["1"][0], outs["0"][0])
+
+
 def test_forward_fp8_empty_batch_and_rejections():
     p = moe.MoEProblem.from_config(SMALL, T=0)
     ws = moe.alloc_workspace(moe.MoEProblem.from_config(SMALL, T=1), moe.MOE_CALL_FORWARD_FP8)
