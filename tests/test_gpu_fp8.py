@@ -174,6 +174,20 @@ def test_forward_fp8_row_gather_and_permuted_copy_agree(monkeypatch, shape):
     assert torch.equal(outs["1"][0], outs["0"][0])
 
 
+@pytest.mark.parametrize("env", [
+    {"MOE_NMAX": "256", "MOE_FUSED_GATHER": "1"},        # E4M3 gather warps on 256-row tiles
+    {"MOE_NMAX": "64", "MOE_DOWN_MB": "1"},              # narrow tiles, one down sub-tile
+])
+def test_forward_fp8_tile_shape_variants(monkeypatch, env):
+    """Forced tile shapes of the FP8 expert GEMMs against the oracle."""
+    for k_, v_ in env.items():
+        monkeypatch.setenv(k_, v_)
+    inp = make_inputs(SMALL, seed=13, device=DEV)
+    cpu = to_cpu_inputs(inp)
+    out, idx, w, _, _ = run_fp8(SMALL, inp)
+    oracle_fp8_parity(SMALL, cpu, out, idx, w, list(range(SMALL.T)))
+
+
 def test_forward_fp8_empty_batch_and_rejections():
     p = moe.MoEProblem.from_config(SMALL, T=0)
     ws = moe.alloc_workspace(moe.MoEProblem.from_config(SMALL, T=1), moe.MOE_CALL_FORWARD_FP8)

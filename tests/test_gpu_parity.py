@@ -362,6 +362,27 @@ def test_forward_gather_variants_agree():
         assert r.returncode == 0 and "ok" in r.stdout, (env, r.stdout[-2000:], r.stderr[-2000:])
 
 
+@pytest.mark.parametrize("env", [
+    {"MOE_NMAX": "64"},                                  # 2 chunks per epilogue warp
+    {"MOE_NMAX": "32", "MOE_DOWN_NMAX": "16"},           # down tile narrower than gate/up
+    {"MOE_NMAX": "256"},                                 # two TMEM batches per sub-tile
+    {"MOE_NMAX": "256", "MOE_FUSED_GATHER": "1"},        # gather warps on 256-row tiles
+    {"MOE_DOWN_MB": "1"},                                # one 128-row sub-tile per down tile
+    {"MOE_NMAX": "160", "MOE_DOWN_MB": "1", "MOE_COMBINE": "atomic"},
+])
+def test_forward_tile_shape_variants(monkeypatch, env):
+    """Forced token-tile widths and down sub-tile counts (the switches are read
+    at every call): each selects another instantiation of the expert GEMMs'
+    epilogue (chunks per warp, TMEM batches per sub-tile, accumulator buffers)
+    on a layer whose experts hold ragged numbers of rows, against the oracle."""
+    for k_, v_ in env.items():
+        monkeypatch.setenv(k_, v_)
+    c = cfg(T=300, H=512, E=16, k=4, I=384)
+    inp = make_inputs(c, seed=21, device=DEV)
+    out, idx, w = run_forward(c, inp)
+    forward_parity(inp, c, out, idx, w)
+
+
 def test_forward_cta_pair_variant():
     """Expert GEMMs run as CTA pairs (MOE_PAIR=1: cta_group::2 MMAs of
     M = 256, each CTA loading half of the token tile): bf16 layers with an odd
