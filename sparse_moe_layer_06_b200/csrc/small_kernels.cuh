@@ -428,11 +428,10 @@ __global__ void combine_kernel(const T* __restrict__ y_perm, const int32_t* __re
 // Fixed-order combine of weighted expert rows (the down GEMM already applied
 // the routing weights): out[t] = sum_j y[pos[t,j]] (j = 0..k-1 in slot order)
 // + y[shared_row0 + t] when shared_row0 >= 0, summed in fp32.  One warp per
-// (token, segment of 64 16-byte vectors of H): two vectors per lane in flight
-// per row, so even a few tokens spread over many warps.  y is bf16 (8 values
-// per vector) or fp32 (4 values per vector).
-constexpr int kSegVecs = 64;  // 16-byte vectors per warp segment
-
+// (token, segment of 32*kVPL 16-byte vectors of H), each lane kVPL vectors of
+// each row; kBatch rows' loads are in flight before any is added (the sums
+// stay in slot order), so even a few tokens spread over many warps.  y is
+// bf16 (8 values per vector) or fp32 (4 values per vector).
 template <typename TIn>
 __device__ __forceinline__ void add_vec(float (&acc)[16 / sizeof(TIn)], const uint4& q) {
     if constexpr (sizeof(TIn) == 2) {
@@ -451,14 +450,15 @@ __device__ __forceinline__ void add_vec(float (&acc)[16 / sizeof(TIn)], const ui
     }
 }
 
-template <typename TIn, typename TOut, int kBatch>
+template <typename TIn, typename TOut, int kBatch, int kVPL>
 __global__ void gather_sum_kernel(const TIn* __restrict__ y, const int32_t* __restrict__ pos,
                                   int64_t T, int H, int k, int64_t n_rows, int64_t shared_row0,
                                   TOut* __restrict__ out, int32_t* status) {
     constexpr int kVE = 16 / static_cast<int>(sizeof(TIn));  // values per 16-byte vector
+    constexpr int kSeg = 32 * kVPL;                           // vectors per warp segment
     const int lane = threadIdx.x & 31;
     const int nvec = H / kVE;
-    const int nseg = (nvec + kSegVecs - 1) / kSegVecs;
+    const int nseg = (nvec + kSeg - 1) / kSeg;
     ptx::grid_dep_wait();  // the rows come from the previous launch
     const int64_t gw = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int64_t t = gw / nseg;
@@ -472,58 +472,61 @@ __global__ void gather_sum_kernel(const TIn* __restrict__ y, const int32_t* __re
     }
     const uint4* yv = reinterpret_cast<const uint4*>(y);
     const int64_t row_vecs = nvec;
-    {
-        const int v0 = seg * kSegVecs;
-        const int va = v0 + lane, vb = v0 + 32 + lane;
-        const bool oka = va < nvec, okb = vb < nvec;
-        float acc_a[kVE], acc_b[kVE];
+    int vi[kVPL];
+    bool ok[kVPL];
+    float acc[kVPL][kVE];
 #pragma unroll
-        for (int e = 0; e < kVE; ++e) acc_a[e] = acc_b[e] = 0.0f;
-        // rows in slot order (the shared expert's last), loaded kBatch at a
-        // time before any is added; the additions stay in slot order
-        const int n_rows_t = k + (shared_row0 >= 0 ? 1 : 0);
-        for (int j0 = 0; j0 < n_rows_t; j0 += kBatch) {
-            uint4 qa[kBatch], qb[kBatch];
-            bool has[kBatch];
+    for (int u = 0; u < kVPL; ++u) {
+        vi[u] = seg * kSeg + 32 * u + lane;
+        ok[u] = vi[u] < nvec;
 #pragma unroll
-            for (int b = 0; b < kBatch; ++b) {
-                const int j = j0 + b;
-                int64_t r = -1;
-                if (j < k) r = __shfl_sync(0xffffffffu, my_pos, j & 31);
-                else if (j < n_rows_t) r = shared_row0 + t;
-                has[b] = r >= 0;
-                if (has[b] && oka) qa[b] = yv[r * row_vecs + va];
-                if (has[b] && okb) qb[b] = yv[r * row_vecs + vb];
-            }
+        for (int e = 0; e < kVE; ++e) acc[u][e] = 0.0f;
+    }
+    // rows in slot order (the shared expert's last)
+    const int n_rows_t = k + (shared_row0 >= 0 ? 1 : 0);
+    for (int j0 = 0; j0 < n_rows_t; j0 += kBatch) {
+        uint4 q[kBatch][kVPL];
+        bool has[kBatch];
 #pragma unroll
-            for (int b = 0; b < kBatch; ++b) {
-                if (has[b] && oka) add_vec<TIn>(acc_a, qa[b]);
-                if (has[b] && okb) add_vec<TIn>(acc_b, qb[b]);
-            }
+        for (int b = 0; b < kBatch; ++b) {
+            const int j = j0 + b;
+            int64_t r = -1;
+            if (j < k) r = __shfl_sync(0xffffffffu, my_pos, j & 31);
+            else if (j < n_rows_t) r = shared_row0 + t;
+            has[b] = r >= 0;
+#pragma unroll
+            for (int u = 0; u < kVPL; ++u)
+                if (has[b] && ok[u]) q[b][u] = yv[r * row_vecs + vi[u]];
         }
-        auto put = [&](const float (&acc)[kVE], int v) {
-            TOut* o = out + t * H + static_cast<int64_t>(v) * kVE;
-            if constexpr (sizeof(TOut) == 2 && kVE == 8) {
-                uint4 q;
-                __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&q);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) h2[e] = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
-                *reinterpret_cast<uint4*>(o) = q;
-            } else if constexpr (sizeof(TOut) == 2) {
-                uint2 q;
-                __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&q);
-                h2[0] = __floats2bfloat162_rn(acc[0], acc[1]);
-                h2[1] = __floats2bfloat162_rn(acc[2], acc[3]);
-                *reinterpret_cast<uint2*>(o) = q;
-            } else {
+        for (int b = 0; b < kBatch; ++b) {
 #pragma unroll
-                for (int e = 0; e < kVE; e += 4)
-                    *reinterpret_cast<float4*>(o + e) =
-                        make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
-            }
-        };
-        if (oka) put(acc_a, va);
-        if (okb) put(acc_b, vb);
+            for (int u = 0; u < kVPL; ++u)
+                if (has[b] && ok[u]) add_vec<TIn>(acc[u], q[b][u]);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < kVPL; ++u) {
+        if (!ok[u]) continue;
+        TOut* o = out + t * H + static_cast<int64_t>(vi[u]) * kVE;
+        if constexpr (sizeof(TOut) == 2 && kVE == 8) {
+            uint4 qo;
+            __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&qo);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) h2[e] = __floats2bfloat162_rn(acc[u][2 * e], acc[u][2 * e + 1]);
+            *reinterpret_cast<uint4*>(o) = qo;
+        } else if constexpr (sizeof(TOut) == 2) {
+            uint2 qo;
+            __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&qo);
+            h2[0] = __floats2bfloat162_rn(acc[u][0], acc[u][1]);
+            h2[1] = __floats2bfloat162_rn(acc[u][2], acc[u][3]);
+            *reinterpret_cast<uint2*>(o) = qo;
+        } else {
+#pragma unroll
+            for (int e = 0; e < kVE; e += 4)
+                *reinterpret_cast<float4*>(o + e) =
+                    make_float4(acc[u][e], acc[u][e + 1], acc[u][e + 2], acc[u][e + 3]);
+        }
     }
 }
 
