@@ -278,7 +278,8 @@ int32_t moe_router_stats(const moe_problem* problem, const void* x, const void* 
  * moe_quantize_weights_fp8 -- encode [n_experts, 3, I, H] weights (problem
  * dtype; device) into E4M3 codes q (same shape, uint8, device) with scales
  * scale_gu [n_experts, 2, I] (gate rows, then up rows) and scale_d
- * [n_experts, H] (fp32, device).  H and I must be multiples of 128.
+ * [n_experts, H] (fp32, device).  H and I must be multiples of 128; w and q
+ * must be 16-byte aligned (else MOE_ERR_INVALID_ARG).
  * Run once per weight set (e.g. at load time); nothing is allocated.
  */
 int32_t moe_quantize_weights_fp8(const moe_problem* problem, int32_t n_experts, const void* w,

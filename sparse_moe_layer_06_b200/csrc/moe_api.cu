@@ -1479,6 +1479,8 @@ int32_t moe_quantize_weights_fp8(const moe_problem* p, int32_t n_experts, const 
                                  uint8_t* q, float* scale_gu, float* scale_d, void* stream) {
     MOE_TRY(check_problem(p));
     if (!w || !q || !scale_gu || !scale_d) return MOE_ERR_INVALID_ARG;
+    // the row encoder reads 16-byte vectors of w and writes 8-byte groups of q
+    if (!aligned16(w) || !aligned16(q)) return MOE_ERR_INVALID_ARG;
     if (n_experts < 1) return MOE_ERR_INVALID_ARG;
     if (p->H % 128 != 0 || p->I % 128 != 0) return MOE_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -585,25 +585,85 @@ __device__ __forceinline__ float load_f32<__nv_bfloat16>(const __nv_bfloat16* p,
 // Row r of the output is row (r / group) * src_group_stride + r % group of the
 // input (group = src_group_stride: plain rows; group = 2*I, stride 3*I: the
 // gate and up rows of [E,3,I,H] expert weights); codes keep the input's layout.
+// len is a multiple of 128 (so rows are 16-byte aligned): each lane reads
+// 16-byte vectors (8 bf16 or 4 fp32 values), eight in flight, and writes each
+// vector's codes at once.
+template <typename T>
+__device__ __forceinline__ void unpack_vec(const uint4& q, float (&f)[16 / sizeof(T)]) {
+    if constexpr (sizeof(T) == 2) {
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 v = __bfloat1622float2(h2[e]);
+            f[2 * e] = v.x;
+            f[2 * e + 1] = v.y;
+        }
+    } else {
+        f[0] = __uint_as_float(q.x);
+        f[1] = __uint_as_float(q.y);
+        f[2] = __uint_as_float(q.z);
+        f[3] = __uint_as_float(q.w);
+    }
+}
+
 template <typename T>
 __global__ void quantize_rows_e4m3_kernel(const T* __restrict__ in, int64_t n_rows, int len,
                                           int64_t group, int64_t src_group_stride,
                                           uint8_t* __restrict__ q, float* __restrict__ scale) {
+    constexpr int kVE = 16 / static_cast<int>(sizeof(T));  // values per 16-byte vector
     const int lane = threadIdx.x & 31;
     const int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (r >= n_rows) return;
     const int64_t src_row = (r / group) * src_group_stride + r % group;
-    const T* row = in + src_row * len;
+    const uint4* row = reinterpret_cast<const uint4*>(in + src_row * len);
+    const int nv = len / kVE;
+    constexpr int kU = 8;  // vectors per lane in flight before any is used
     float amax = 0.0f;
-    for (int i = lane; i < len; i += 32) amax = fmaxf(amax, fabsf(load_f32(row, i)));
+    for (int v0 = lane; v0 < nv; v0 += 32 * kU) {
+        uint4 qv[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u)
+            if (v0 + 32 * u < nv) qv[u] = row[v0 + 32 * u];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            if (v0 + 32 * u < nv) {
+                float f[kVE];
+                unpack_vec<T>(qv[u], f);
+#pragma unroll
+                for (int e = 0; e < kVE; ++e) amax = fmaxf(amax, fabsf(f[e]));
+            }
+        }
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     const float sc = pow2_scale_f(amax);
     const float inv = 1.0f / sc;  // exact: power of two
     uint8_t* qr = q + src_row * len;
-    for (int i = 2 * lane; i < len; i += 64) {
-        const uint16_t two = ptx::e4m3x2(load_f32(row, i) * inv, load_f32(row, i + 1) * inv);
-        *reinterpret_cast<uint16_t*>(qr + i) = two;
+    for (int v0 = lane; v0 < nv; v0 += 32 * kU) {
+        uint4 qv[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u)
+            if (v0 + 32 * u < nv) qv[u] = row[v0 + 32 * u];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int v = v0 + 32 * u;
+            if (v < nv) {
+                float f[kVE];
+                unpack_vec<T>(qv[u], f);
+                uint32_t c[kVE / 4];
+#pragma unroll
+                for (int w = 0; w < kVE / 4; ++w)
+                    c[w] = static_cast<uint32_t>(ptx::e4m3x2(f[4 * w] * inv, f[4 * w + 1] * inv)) |
+                           (static_cast<uint32_t>(
+                                ptx::e4m3x2(f[4 * w + 2] * inv, f[4 * w + 3] * inv))
+                            << 16);
+                if constexpr (kVE == 8)
+                    *reinterpret_cast<uint2*>(qr + static_cast<int64_t>(v) * kVE) =
+                        make_uint2(c[0], c[1]);
+                else
+                    *reinterpret_cast<uint32_t*>(qr + static_cast<int64_t>(v) * kVE) = c[0];
+            }
+        }
     }
     if (lane == 0) scale[r] = sc;
 }

@@ -132,6 +132,24 @@ def test_ffn_and_permute_validation(lib):
                          None) == moe.MOE_ERR_WORKSPACE
 
 
+def test_fp8_weight_encoder_validation(lib):
+    # fake, never-dereferenced addresses: refused on the host before any launch
+    # (the row encoder reads 16-byte vectors of w and writes 8-byte groups of q)
+    p = problem(H=256, I=256).c()
+    P = ctypes.c_void_p
+    a = 1 << 20
+    before = moe.moe_launch_count()
+
+    def enc(pc, n, w, q):
+        return lib.moe_quantize_weights_fp8(ctypes.byref(pc), n, P(w), P(q), P(a), P(a), None)
+
+    assert enc(p, 2, a + 2, a) == moe.MOE_ERR_INVALID_ARG      # w not 16-byte aligned
+    assert enc(p, 2, a, a + 8) == moe.MOE_ERR_INVALID_ARG      # q not 16-byte aligned
+    assert enc(p, 0, a, a) == moe.MOE_ERR_INVALID_ARG          # no experts
+    assert enc(problem(H=192, I=256).c(), 2, a, a) == moe.MOE_ERR_UNSUPPORTED
+    assert moe.moe_launch_count() == before
+
+
 def test_binding_refuses_cpu_tensors(lib):
     p = problem(T=4, H=64, I=64, E=2, top_k=1, num_shared=0)
     x = torch.zeros(4, 64, dtype=torch.bfloat16)
