@@ -35,8 +35,10 @@ from sparse_moe_layer_06_b200.workloads import CONFIGS, make_inputs, make_x, sam
 
 METRIC = "MoE-layer tokens/s and % of roofline (TFLOP/s or HBM GB/s) on 1 B200"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# the expert GEMM kernels and their launch configuration (template arguments)
 GEMM_SOURCES = ["sparse_moe_layer_06_b200/csrc/gemm_sm100.cuh",
-                "sparse_moe_layer_06_b200/csrc/ptx.cuh"]
+                "sparse_moe_layer_06_b200/csrc/ptx.cuh",
+                "sparse_moe_layer_06_b200/csrc/moe_api.cu"]
 
 
 # ------------------------------------------------------------------ helpers

@@ -532,6 +532,13 @@ int32_t launch_gemm_n(const GemmArgs& a, int grid, cudaStream_t s, const char* n
 // rows.  Off by default: the pairs halve the token-tile reads from L2 but
 // measured slower at the Hy4 prefill shapes (the two CTAs advance in
 // lockstep), and only about 1% faster on the tensor-bound skewed batch.
+// Warps that gather the gate/up GEMM's token rows (the fused row gather).
+// Three measured 1-3% faster per prefill layer than four (bf16 and FP8; Hy3
+// 1%; decode unchanged) and two slower: with fewer warps, fewer of them
+// compete with the epilogue for the shared-memory pipe, while three still keep
+// the token-row stages ahead of the MMAs.
+constexpr int kGatherWarps = 3;
+
 bool use_pair() {
     const bool v = env_int("MOE_PAIR", 0) != 0;
     return v;
@@ -567,14 +574,14 @@ int32_t launch_gemm_fp8(int nmax, int mb, const GemmArgs& a, int64_t max_tiles, 
     const bool pair = use_pair() && nmax >= 64;
     if constexpr (EPI == EPI_SWIGLU) {
         if (a.gather_tok != nullptr) {
-            // E4M3 token rows gathered by four gather warps
+            // E4M3 token rows gathered by the gather warps
             switch (nmax) {
-                case 16: return launch_gemm_n<EPI, 16, 2, 1, false, 4>(a, grid, s, name, false, pdl);
-                case 32: return launch_gemm_n<EPI, 32, 2, 1, false, 4>(a, grid, s, name, false, pdl);
-                case 64: return launch_gemm_n<EPI, 64, 2, 1, false, 4>(a, grid, s, name, false, pdl);
-                case 128: return launch_gemm_n<EPI, 128, 2, 1, false, 4>(a, grid, s, name, false, pdl);
-                case 160: return launch_gemm_n<EPI, 160, 2, 1, false, 4>(a, grid, s, name, false, pdl);
-                case 256: return launch_gemm_n<EPI, 256, 2, 1, false, 4>(a, grid, s, name, false, pdl);
+                case 16: return launch_gemm_n<EPI, 16, 2, 1, false, kGatherWarps>(a, grid, s, name, false, pdl);
+                case 32: return launch_gemm_n<EPI, 32, 2, 1, false, kGatherWarps>(a, grid, s, name, false, pdl);
+                case 64: return launch_gemm_n<EPI, 64, 2, 1, false, kGatherWarps>(a, grid, s, name, false, pdl);
+                case 128: return launch_gemm_n<EPI, 128, 2, 1, false, kGatherWarps>(a, grid, s, name, false, pdl);
+                case 160: return launch_gemm_n<EPI, 160, 2, 1, false, kGatherWarps>(a, grid, s, name, false, pdl);
+                case 256: return launch_gemm_n<EPI, 256, 2, 1, false, kGatherWarps>(a, grid, s, name, false, pdl);
                 default: return MOE_ERR_UNSUPPORTED;
             }
         }
@@ -607,14 +614,14 @@ int32_t launch_gemm(int nmax, int mb, const GemmArgs& a, int64_t max_tiles, cuda
     int grid = static_cast<int>(std::min<int64_t>(sm_count(), std::max<int64_t>(1, max_tiles)));
     if constexpr (EPI == EPI_SWIGLU) {
         if (a.gather_tok != nullptr) {
-            // row gather by four dedicated gather warps
+            // row gather by the dedicated gather warps
             switch (nmax) {
-                case 16: return launch_gemm_n<EPI, 16, 2, 0, false, 4>(a, grid, s, name, false, pdl);
-                case 32: return launch_gemm_n<EPI, 32, 2, 0, false, 4>(a, grid, s, name, false, pdl);
-                case 64: return launch_gemm_n<EPI, 64, 2, 0, false, 4>(a, grid, s, name, false, pdl);
-                case 128: return launch_gemm_n<EPI, 128, 2, 0, false, 4>(a, grid, s, name, false, pdl);
-                case 160: return launch_gemm_n<EPI, 160, 2, 0, false, 4>(a, grid, s, name, false, pdl);
-                case 256: return launch_gemm_n<EPI, 256, 2, 0, false, 4>(a, grid, s, name, false, pdl);
+                case 16: return launch_gemm_n<EPI, 16, 2, 0, false, kGatherWarps>(a, grid, s, name, false, pdl);
+                case 32: return launch_gemm_n<EPI, 32, 2, 0, false, kGatherWarps>(a, grid, s, name, false, pdl);
+                case 64: return launch_gemm_n<EPI, 64, 2, 0, false, kGatherWarps>(a, grid, s, name, false, pdl);
+                case 128: return launch_gemm_n<EPI, 128, 2, 0, false, kGatherWarps>(a, grid, s, name, false, pdl);
+                case 160: return launch_gemm_n<EPI, 160, 2, 0, false, kGatherWarps>(a, grid, s, name, false, pdl);
+                case 256: return launch_gemm_n<EPI, 256, 2, 0, false, kGatherWarps>(a, grid, s, name, false, pdl);
                 default: return MOE_ERR_UNSUPPORTED;
             }
         }
@@ -660,7 +667,7 @@ bool combine_atomic() {
 }
 
 // Whether the gate/up GEMM gathers the routed token rows straight from x
-// (four gather warps, 16-byte cp.async into the swizzled stage; bf16 rows,
+// (kGatherWarps gather warps, 16-byte cp.async into the swizzled stage; bf16 rows,
 // or the E4M3 code rows of moe_forward_fp8) instead of reading a permuted copy
 // x_perm written by a separate
 // gather kernel.  Default: fused for token tiles of up to 160 rows (measured
